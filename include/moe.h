@@ -1,0 +1,200 @@
+/*
+ * C ABI of the B200 routed Mixture-of-Experts layer forward (sm_100a).
+ *
+ * The layer (NeMo AutoModel "Step-5-Preview" page, "Model Architecture" table):
+ * hidden H = 4,096; a learned router over E = 352 routed experts with top-k = 8
+ * routing and one always-on shared expert; every expert a SwiGLU MLP with
+ * intermediate size I = 1,536. Expert weights are BF16, or FP8 E4M3 with one
+ * fp32 scale per 128x128 block (StepFun "Step-5 minimal inference" README:
+ * "block-scaled FP8 expert GEMM"; expert storage follows the checkpoint's
+ * quantization_config). The MoE primitives around the expert GEMMs (routing,
+ * the token->expert histogram and permutation, the combine) are the same
+ * README's "critical MoE primitives".
+ *
+ * What one call computes, per token t:
+ *   l      = x[t] . Wr^T (+ b)                 fp32 logits over the E experts
+ *   top-k  = the k largest logits, ties to the lower expert index,
+ *            in descending order; g = softmax(l) over the chosen k, renormalised
+ *   y_e    = (silu(a W1_e^T) * (a W3_e^T)) W2_e^T   for the k chosen experts
+ *            and the shared expert; a = x[t] (BF16 storage) or its 1x128-block
+ *            E4M3 quantisation (FP8 storage: scale = blockmax/448)
+ *   out[t] = sum_j g_j y_{e_j} + y_shared      summed in fp32 in slot order,
+ *                                              rounded once to bf16
+ *
+ * Conventions for every entry point:
+ *  - Layouts are row-major and C-contiguous. Weights are in nn.Linear order
+ *    ([out, in], the reduction dimension contiguous):
+ *      router_w [E, H] bf16;  w1, w3 [E, I, H];  w2 [E, H, I];
+ *      FP8 scales s1, s3 [E, I/128, H/128] fp32;  s2 [E, H/128, I/128] fp32;
+ *      the shared expert's sw1, sw3, sw2 (and ss1, ss3, ss2) have the same
+ *      layouts with E = 1.
+ *  - "Device" pointers are CUDA device memory of the current device; the
+ *    caller owns every buffer. The library allocates no device memory: all
+ *    scratch comes from the caller's workspace (size: moe_workspace_bytes).
+ *  - Calls are asynchronous on `stream` unless stated. Argument errors are
+ *    returned synchronously; errors found on the device (a bad expert index,
+ *    a timed-out wait) are latched in a status word inside the workspace and
+ *    read with moe_read_status.
+ *  - Device buffers must be 16-byte aligned (TMA); 256-byte alignment is
+ *    recommended. The workspace must be 1024-byte aligned.
+ *  - Supported shapes: H and I multiples of 128; 1 <= E <= 512;
+ *    1 <= top_k <= min(E, 16); n_shared in {0, 1}; 0 <= T, (top_k+n_shared)*T < 2^31.
+ *    T == 0 is a no-op that returns MOE_OK.
+ */
+#ifndef MOE_B200_H
+#define MOE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define MOE_API __attribute__((visibility("default")))
+#else
+#define MOE_API
+#endif
+
+/* Same object as cudaStream_t; NULL is the legacy default stream. */
+typedef struct CUstream_st* moe_stream_t;
+
+/* Expert weight storage. */
+enum {
+  MOE_WDTYPE_BF16 = 0,     /* bf16 weights, bf16 activations */
+  MOE_WDTYPE_FP8_E4M3 = 1  /* E4M3 weights with 128x128 fp32 block scales, E4M3 1x128 activations */
+};
+
+/* Status codes (returned, or latched on the device). */
+enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1,        /* null pointer, bad config or size */
+  MOE_ERR_UNSUPPORTED_SHAPE = 2,  /* a shape outside the supported set */
+  MOE_ERR_WORKSPACE_TOO_SMALL = 3,
+  MOE_ERR_CUDA = 4,               /* a CUDA runtime call failed (no device, launch error, ...) */
+  MOE_ERR_BAD_INDEX = 5,          /* device: an expert index outside [0, E) was skipped */
+  MOE_ERR_DEVICE_TIMEOUT = 6,     /* device: a bounded wait gave up; results are invalid */
+  MOE_ERR_MISALIGNED = 7          /* a buffer is not 16-byte (workspace: 1024-byte) aligned */
+};
+
+typedef struct moe_config {
+  int32_t hidden;     /* H */
+  int32_t n_experts;  /* E, routed experts */
+  int32_t top_k;      /* k */
+  int32_t n_shared;   /* 0 or 1 always-on shared expert */
+  int32_t inter;      /* I, expert intermediate size */
+  int32_t wdtype;     /* MOE_WDTYPE_* */
+} moe_config;
+
+/* Device pointers to one layer's weights (see the layouts above). Scale
+ * pointers are used only for MOE_WDTYPE_FP8_E4M3; shared-expert pointers only
+ * when n_shared == 1. router_bias may be NULL (no bias). */
+typedef struct moe_weights {
+  const void* router_w;
+  const float* router_bias;
+  const void* w1;
+  const void* w3;
+  const void* w2;
+  const float* s1;
+  const float* s3;
+  const float* s2;
+  const void* sw1;
+  const void* sw3;
+  const void* sw2;
+  const float* ss1;
+  const float* ss3;
+  const float* ss2;
+} moe_weights;
+
+/* Bytes of workspace that moe_forward (and every stage entry point) needs for
+ * T tokens. Host only; touches no device. */
+MOE_API int moe_workspace_bytes(const moe_config* cfg, int64_t T, size_t* bytes);
+
+/*
+ * The whole layer forward: router + top-k, histogram/scan/permute, grouped
+ * expert GEMMs (gate/up with fused SwiGLU, then down), combine.
+ *   x        [T, H] bf16, device
+ *   out      [T, H] bf16, device (written)
+ *   topk_idx [T, k] int32 and topk_w [T, k] fp32, device, optional (NULL): if
+ *            given, the routing decision is written there as well.
+ */
+MOE_API int moe_forward(const moe_config* cfg, int64_t T, const void* x, const moe_weights* w, void* out,
+                int32_t* topk_idx, float* topk_w, void* workspace, size_t workspace_bytes,
+                moe_stream_t stream);
+
+/*
+ * moe_forward from host memory: copies x_host [T, H] bf16 to the device,
+ * runs the layer and copies the result into out_host [T, H] bf16; weights and
+ * workspace are device memory. Synchronous: returns after out_host is written
+ * (pinned host buffers make the copies asynchronous DMA).
+ */
+MOE_API int moe_forward_host(const moe_config* cfg, int64_t T, const void* x_host, const moe_weights* w,
+                     void* out_host, void* workspace, size_t workspace_bytes, moe_stream_t stream);
+
+/* ---- stage entry points (each a part of moe_forward, for tests and tools) ---- */
+
+/* Router: fp32 logits, top-k selection and renormalised gates.
+ * logits [T, E] fp32 (optional): the fp32 logits including the bias. */
+MOE_API int moe_route(const moe_config* cfg, int64_t T, const void* x, const void* router_w,
+              const float* router_bias, int32_t* topk_idx, float* topk_w, float* logits,
+              void* workspace, size_t workspace_bytes, moe_stream_t stream);
+
+/* Activation quantisation of x [T, H] bf16 into E4M3 codes q [T, H] and fp32
+ * scales s [T, H/128] (one per 1x128 row block, scale = blockmax/448; an
+ * all-zero block gets scale 1 and zero codes). */
+MOE_API int moe_quantize_act(int64_t T, int32_t hidden, const void* x, uint8_t* q, float* s, moe_stream_t stream);
+
+/* Histogram/scan/permute of a routing decision. Groups 0..E-1 are the routed
+ * experts, group E the shared expert (all T tokens) when n_shared == 1.
+ *   counts  [E+S] int32    rows per group
+ *   offsets [E+S+1] int32  exclusive scan of counts
+ *   perm    [(k+S)T] int32 token of each row; rows of a group ascend by token
+ *   pos     [T, k+S] int32 row of (token, slot); slot k is the shared row
+ * An out-of-range index latches MOE_ERR_BAD_INDEX and its pair is skipped. */
+MOE_API int moe_permute(const moe_config* cfg, int64_t T, const int32_t* topk_idx, int32_t* counts,
+                int32_t* offsets, int32_t* perm, int32_t* pos, void* workspace, size_t workspace_bytes,
+                moe_stream_t stream);
+
+/* Expert MLPs for a given routing: permute, gather (+ quantise), gate/up GEMM
+ * with SwiGLU, down GEMM. y [(k+S)T, H] bf16 receives each row's expert output
+ * times its gate (1 for shared rows); pos [T, k+S] receives the row of each
+ * (token, slot). */
+MOE_API int moe_experts(const moe_config* cfg, int64_t T, const void* x, const int32_t* topk_idx,
+                const float* topk_w, const moe_weights* w, void* y, int32_t* pos, void* workspace,
+                size_t workspace_bytes, moe_stream_t stream);
+
+/* Combine: out[t] = sum over slots j < k+S of y[pos[t, j]], fp32 in slot
+ * order, rounded once to bf16. y [(k+S)T, H] bf16, pos [T, k+S], out [T, H]. */
+MOE_API int moe_combine(const moe_config* cfg, int64_t T, const void* y, const int32_t* pos, void* out,
+                moe_stream_t stream);
+
+/* ---- status and profiling ---- */
+
+/* Synchronises `stream`, then returns the device status latched in the
+ * workspace since the last moe_* call that cleared it (every moe_forward,
+ * moe_route, moe_permute and moe_experts call clears it first). */
+MOE_API int moe_read_status(const void* workspace, moe_stream_t stream, int* device_status);
+
+/* Text for a status code (static storage). */
+MOE_API const char* moe_status_string(int status);
+
+/* Per-kernel timing of moe_forward: when enabled, moe_forward records a CUDA
+ * event before and after each of its kernels on its stream. */
+MOE_API int moe_profile_enable(int enable);
+
+/* Synchronises on the last recorded event and writes the kernel times (ms) of
+ * the most recent profiled moe_forward into ms[0..n); *n_out = number of
+ * kernels. Names come from moe_profile_kernel_name. */
+MOE_API int moe_profile_read(float* ms, int n, int* n_out);
+MOE_API const char* moe_profile_kernel_name(int i);
+
+/* Number of streaming multiprocessors the kernels size their grids for
+ * (current device). */
+MOE_API int moe_device_sm_count(int* sms);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_B200_H */

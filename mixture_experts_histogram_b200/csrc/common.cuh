@@ -1,0 +1,121 @@
+// Shared declarations of the CUDA library: kernel parameter blocks, the
+// workspace layout, and the host-side launch functions of each kernel family.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "moe.h"
+
+namespace moe {
+
+constexpr int kTileM = 128;          // rows (tokens) per expert-GEMM tile
+constexpr int kStageBytesK = 128;    // K extent of one pipeline stage, in bytes (one 128B swizzle row)
+constexpr int kHistChunk = 256;      // tokens per histogram/scatter CTA
+constexpr int kMaxExperts = 512;
+constexpr int kMaxTopK = 16;
+
+__host__ __device__ inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+__host__ __device__ inline int64_t round_up(int64_t a, int64_t b) { return ceil_div(a, b) * b; }
+
+// Where each scratch buffer lives inside the caller's workspace (byte offsets
+// from its base; every buffer starts on a 1024-byte boundary).
+struct WsLayout {
+  int64_t T, R, rows_pad, chunks, ksplit;
+  size_t status, idx, gate, logits_part, chunk_base, counts, offsets, mt_prefix;
+  size_t perm, pos, row_gate, xp, sxp, h, sh, y, x_stage, out_stage, total;
+};
+
+WsLayout ws_layout(const moe_config& c, int64_t T, int num_sms);
+
+// ---- router (logits GEMM on tcgen05 + top-k/softmax) ----
+struct RouterParams {
+  int32_t T, H, E;
+  int32_t nbox;         // B boxes per stage (1 or 2)
+  int32_t box_rows;     // rows per B box (multiple of 16, <= 256)
+  int32_t ksplit;       // K splits (grid.y)
+  int32_t kstages;      // total K stages (H / 64)
+  float* partial;       // [ksplit, T, E] fp32
+  int* status;
+};
+
+struct TopkParams {
+  int32_t T, E, k, ksplit;
+  const float* partial;     // [ksplit, T, E]
+  const float* bias;        // [E] or null
+  int32_t* idx;             // [T, k]
+  float* gate;              // [T, k]
+  float* logits;            // [T, E] or null
+};
+
+// ---- histogram / scan / scatter ----
+struct PermuteParams {
+  int32_t T, E, k, S, G, chunks;
+  const int32_t* idx;       // [T, k]
+  const float* gate;        // [T, k] or null (row gates then not written)
+  int32_t* chunk_base;      // [E, chunks]: per-chunk counts, then absolute row bases
+  int32_t* counts;          // [G]
+  int32_t* offsets;         // [G + 1]
+  int32_t* mt_prefix;       // [G + 1] M-tile prefix (tiles of kTileM rows)
+  int32_t* perm;            // [S T]
+  int32_t* pos;             // [T, S]
+  float* row_gate;          // [S T] or null
+  int* status;
+};
+
+// ---- gather (+ E4M3 quantisation) ----
+struct GatherParams {
+  int32_t T, H, S;
+  int64_t rows_pad;         // row stride of the transposed scale array
+  const uint16_t* x;        // [T, H] bf16
+  const int32_t* pos;       // [T, S] destination rows (null: row = token, S = 1)
+  void* xp;                 // [rows, H] bf16 or E4M3
+  float* sxp;               // FP8: scales, [H/128, rows_pad] (transposed) or [T, H/128]
+  int32_t scale_row_major;  // 1: scales stored [T, H/128]
+};
+
+// ---- grouped expert GEMMs ----
+struct GemmParams {
+  const int32_t* mt_prefix;  // [G + 1]
+  const int32_t* offsets;    // [G + 1]
+  int32_t G, E;              // groups, routed experts (group E is the shared expert)
+  int32_t K, N;              // reduction length; output width (I for GEMM1, H for GEMM2)
+  int32_t n_tiles;           // output tiles per M tile
+  int32_t R;                 // total rows
+  int64_t rows_pad;          // row stride of transposed activation scales
+  const float* a_scale;      // FP8: [K/128, rows_pad]
+  const float* b_scale0;     // FP8 routed scales (GEMM1: s1, GEMM2: s2)
+  const float* b_scale1;     // FP8 routed scales (GEMM1: s3)
+  const float* bs_scale0;    // FP8 shared-expert scales
+  const float* bs_scale1;
+  void* out;                 // GEMM1: h [R, N]; GEMM2: y [R, N] bf16
+  float* out_scale;          // GEMM1 FP8: [N/128, rows_pad]
+  const float* row_gate;     // GEMM2: [R]
+  int* status;
+};
+
+struct CombineParams {
+  int32_t T, H, S;
+  const uint16_t* y;         // [S T, H] bf16
+  const int32_t* pos;        // [T, S]
+  uint16_t* out;             // [T, H] bf16
+};
+
+// Host launchers (each returns the launch's cudaError_t).
+cudaError_t launch_router_gemm(const RouterParams& p, const CUtensorMap& tm_x, const CUtensorMap& tm_w,
+                               cudaStream_t s);
+cudaError_t launch_topk(const TopkParams& p, cudaStream_t s);
+cudaError_t launch_histogram(const PermuteParams& p, cudaStream_t s);
+cudaError_t launch_scan(const PermuteParams& p, cudaStream_t s);
+cudaError_t launch_scatter(const PermuteParams& p, cudaStream_t s);
+cudaError_t launch_gather(const GatherParams& p, bool fp8, cudaStream_t s);
+cudaError_t launch_gemm1(const GemmParams& p, bool fp8, int grid, const CUtensorMap& tm_a,
+                         const CUtensorMap& tm_w1, const CUtensorMap& tm_w3, const CUtensorMap& tm_sw1,
+                         const CUtensorMap& tm_sw3, cudaStream_t s);
+cudaError_t launch_gemm2(const GemmParams& p, bool fp8, int grid, const CUtensorMap& tm_a,
+                         const CUtensorMap& tm_w2, const CUtensorMap& tm_sw2, cudaStream_t s);
+cudaError_t launch_combine(const CombineParams& p, cudaStream_t s);
+
+}  // namespace moe

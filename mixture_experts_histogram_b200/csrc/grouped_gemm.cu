@@ -1,0 +1,434 @@
+// Grouped expert GEMMs on the 5th-generation tensor cores (tcgen05 + TMEM + TMA).
+//
+// The experts are SwiGLU MLPs (NeMo AutoModel "Step-5-Preview" page, "Model
+// Architecture": 352 routed experts and one shared expert, intermediate size
+// 1,536); expert weights are BF16 or block-scaled FP8 E4M3 (StepFun "Step-5
+// minimal inference" README: "block-scaled FP8 expert GEMM"). The shared
+// expert is simply group E, after the routed groups.
+//
+//   GEMM1 (gate/up + SwiGLU):  for each row r of group g and output column j < I
+//       h[r, j] = silu(A[r] . W1_g[j]) * (A[r] . W3_g[j])
+//     BF16: h stored bf16. FP8: h quantised per 1x128 block (scale = blockmax/448),
+//     codes E4M3, scales stored transposed [I/128, rows].
+//   GEMM2 (down):  y[r, c] = gate[r] * (h[r] . W2_g[c]), stored bf16.
+//
+// Tiles: 128 rows x 256 accumulator columns. GEMM1 puts 128 gate columns (W1
+// rows n0..n0+127) and the matching 128 up columns (W3 rows n0..n0+127) side by
+// side in one N = 256 MMA, so SwiGLU pairs sit in one thread's registers. GEMM2
+// covers 256 output columns.
+//
+// Persistent CTAs (one per SM) walk a static list of work items; an item is
+// (group, N tile, M tile) with the M tiles of one (group, N tile) adjacent, so
+// CTAs that share a weight tile run together and the second read hits L2.
+// Warp roles:
+//   warp 0      TMA producer: A tile (128 rows x 128 B) + B tile (256 rows x 128 B)
+//               per stage into a 4-deep ring (128B swizzle).
+//   warp 1      allocates 512 TMEM columns; one thread issues the MMAs.
+//   warps 2-9   epilogue: each thread owns one row (TMEM lane) and one half of
+//               the tile's columns.
+// BF16: the accumulator lives in TMEM for the whole K loop; two 256-column
+// buffers let the epilogue of one tile overlap the MMAs of the next.
+// FP8: the fp32 block scales are not powers of two, so each 128-deep K block is
+// computed into a TMEM partial (two ping-pong buffers) and the epilogue warps
+// promote it into register accumulators with sa[row, kb] * sb[nblk, kb].
+#include <cuda_bf16.h>
+#include <cuda_fp8.h>
+
+#include "common.cuh"
+#include "ptx.cuh"
+
+namespace moe {
+
+namespace {
+
+constexpr int kThreads = 320;
+constexpr int kStages = 4;
+constexpr int kABytes = kTileM * kStageBytesK;  // 16 KB
+constexpr int kBBytes = 256 * kStageBytesK;     // 32 KB
+constexpr int kStageBytes = kABytes + kBBytes;
+constexpr int kMaxGroups = kMaxExperts + 1;
+
+struct SmemLayout {
+  static constexpr size_t kTiles = (size_t)kStages * kStageBytes;
+  static constexpr size_t kBars = kTiles;                              // full[4], empty[4], tfull[2], tempty[2], drain
+  static constexpr size_t kMisc = kBars + 16 * 8;                      // tmem slot, abort flag
+  static constexpr size_t kAmax = kMisc + 64;                          // float [2][2][128]
+  static constexpr size_t kMt = kAmax + 2 * 2 * 128 * 4;               // int [kMaxGroups + 1]
+  static constexpr size_t kOff = kMt + (kMaxGroups + 1) * 4;           // int [kMaxGroups + 1]
+  static constexpr size_t kEnd = kOff + (kMaxGroups + 1) * 4;
+  static constexpr size_t kDynamic = kEnd + 1024;                      // + alignment slack
+};
+
+struct Item {
+  int g, n, row0, valid;
+};
+
+__device__ __forceinline__ Item decode_item(int item, int n_tiles, int G, const int* s_mt, const int* s_off) {
+  const int q = item / n_tiles;
+  int lo = 0, hi = G;  // s_mt[lo] <= q < s_mt[hi]
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (s_mt[mid] <= q) lo = mid;
+    else hi = mid;
+  }
+  Item it;
+  it.g = lo;
+  const int mtiles = s_mt[lo + 1] - s_mt[lo];
+  const int local = item - n_tiles * s_mt[lo];
+  it.n = local / mtiles;
+  const int m = local % mtiles;
+  it.row0 = s_off[lo] + m * kTileM;
+  it.valid = min(kTileM, s_off[lo + 1] - it.row0);
+  return it;
+}
+
+__device__ __forceinline__ float silu_mul(float g, float u) { return g / (1.0f + __expf(-g)) * u; }
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
+  const __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<const uint32_t*>(&v);
+}
+
+// Bounded wait by every lane, with a warp-uniform verdict (keeps the warp
+// converged for the .sync.aligned TMEM loads that follow).
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, int* status, volatile int* abort_flag) {
+  const bool ok = mbar_wait(bar, parity, status, abort_flag);
+  return __all_sync(0xffffffffu, ok);
+}
+
+template <bool kFP8, bool kGemm1>
+__global__ void __launch_bounds__(kThreads, 1)
+    grouped_gemm_kernel(const GemmParams p, const __grid_constant__ CUtensorMap tm_a,
+                        const __grid_constant__ CUtensorMap tm_b0, const __grid_constant__ CUtensorMap tm_b1,
+                        const __grid_constant__ CUtensorMap tm_bs0, const __grid_constant__ CUtensorMap tm_bs1) {
+  constexpr int kElemsPerStage = kFP8 ? 128 : 64;  // 128 bytes of K per stage
+  constexpr uint32_t kIdesc = idesc_mma(kFP8 ? 0u : 1u, kTileM, 256);
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + kStages * kABytes;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + SmemLayout::kBars);
+  uint64_t* empty = full + kStages;
+  uint64_t* tfull = empty + kStages;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* drain = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + SmemLayout::kMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  float* amax_x = reinterpret_cast<float*>(smem + SmemLayout::kAmax);
+  int* s_mt = reinterpret_cast<int*>(smem + SmemLayout::kMt);
+  int* s_off = reinterpret_cast<int*>(smem + SmemLayout::kOff);
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+
+  for (int i = threadIdx.x; i <= p.G; i += kThreads) {
+    s_mt[i] = p.mt_prefix[i];
+    s_off[i] = p.offsets[i];
+  }
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&tfull[b], 1);
+      mbar_init(&tempty[b], 256);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tm_a);
+    tma_prefetch_desc(&tm_b0);
+    tma_prefetch_desc(&tm_bs0);
+    if (kGemm1) {
+      tma_prefetch_desc(&tm_b1);
+      tma_prefetch_desc(&tm_bs1);
+    }
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  __syncthreads();
+  tc_fence_after_sync();
+  const uint32_t tmem = *tmem_slot;
+  const int total = s_mt[p.G] * p.n_tiles;
+  const int kstages = p.K / kElemsPerStage;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---------------------------------------------------- TMA producer --
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t issued = 0;  // bit s: stage s has a load in flight at phase bit (issued_phase >> s) & 1
+      uint32_t issued_phase = 0;
+      bool ok = true;
+      for (int item = blockIdx.x; item < total && ok; item += gridDim.x) {
+        const Item it = decode_item(item, p.n_tiles, p.G, s_mt, s_off);
+        const bool shared = (it.g == p.E);
+        int yb;
+        if (kGemm1) yb = (shared ? 0 : it.g * p.N) + it.n * 128;
+        else yb = (shared ? 0 : it.g * p.N) + it.n * 256;
+        const CUtensorMap* mb0 = shared ? &tm_bs0 : &tm_b0;
+        const CUtensorMap* mb1 = kGemm1 ? (shared ? &tm_bs1 : &tm_b1) : mb0;
+        for (int ks = 0; ks < kstages; ++ks) {
+          if (!mbar_wait(&empty[stage], phase ^ 1, p.status, abort_flag)) { ok = false; break; }
+          mbar_arrive_expect_tx(&full[stage], kStageBytes);
+          const int kx = ks * kElemsPerStage;
+          tma_load_2d(sA + stage * kABytes, &tm_a, &full[stage], kx, it.row0);
+          tma_load_2d(sB + stage * kBBytes, mb0, &full[stage], kx, yb);
+          tma_load_2d(sB + stage * kBBytes + kBBytes / 2, mb1, &full[stage], kx, kGemm1 ? yb : yb + 128);
+          issued |= 1u << stage;
+          issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
+          if (++stage == kStages) { stage = 0; phase ^= 1; }
+        }
+      }
+      if (!ok) {
+        // Let the copies already in flight land before the CTA leaves.
+        for (int s = 0; s < kStages; ++s) {
+          if (!(issued & (1u << s))) continue;
+          const uint64_t t0 = global_timer_ns();
+          while (!mbar_try_wait(&full[s], (issued_phase >> s) & 1u) && global_timer_ns() - t0 < 200000000ull) {}
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ------------------------------------------------------ MMA issuer --
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t acc_iter = 0;
+      bool ok = true;
+      for (int item = blockIdx.x; item < total && ok; item += gridDim.x) {
+        if (!kFP8) {
+          const uint32_t b = acc_iter & 1u, tph = (acc_iter >> 1) & 1u;
+          if (!mbar_wait(&tempty[b], tph ^ 1u, p.status, abort_flag)) { ok = false; break; }
+          tc_fence_after_sync();
+          const uint32_t d = tmem + b * 256;
+          for (int ks = 0; ks < kstages; ++ks) {
+            if (!mbar_wait(&full[stage], phase, p.status, abort_flag)) { ok = false; break; }
+            tc_fence_after_sync();
+            const uint64_t ad = sdesc_k_sw128(sA + stage * kABytes);
+            const uint64_t bd = sdesc_k_sw128(sB + stage * kBBytes);
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) mma_bf16(d, ad + 2 * kk, bd + 2 * kk, kIdesc, (ks | kk) ? 1u : 0u);
+            mma_commit(&empty[stage]);
+            if (++stage == kStages) { stage = 0; phase ^= 1; }
+          }
+          if (!ok) break;
+          mma_commit(&tfull[b]);
+          ++acc_iter;
+        } else {
+          for (int ks = 0; ks < kstages; ++ks) {
+            const uint32_t b = acc_iter & 1u, tph = (acc_iter >> 1) & 1u;
+            if (!mbar_wait(&tempty[b], tph ^ 1u, p.status, abort_flag)) { ok = false; break; }
+            if (!mbar_wait(&full[stage], phase, p.status, abort_flag)) { ok = false; break; }
+            tc_fence_after_sync();
+            const uint32_t d = tmem + b * 256;
+            const uint64_t ad = sdesc_k_sw128(sA + stage * kABytes);
+            const uint64_t bd = sdesc_k_sw128(sB + stage * kBBytes);
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) mma_e4m3(d, ad + 2 * kk, bd + 2 * kk, kIdesc, kk ? 1u : 0u);
+            mma_commit(&empty[stage]);
+            mma_commit(&tfull[b]);
+            ++acc_iter;
+            if (++stage == kStages) { stage = 0; phase ^= 1; }
+          }
+        }
+      }
+      // Drain: every MMA issued so far has completed once this arrives.
+      mma_commit(drain);
+      const uint64_t t0 = global_timer_ns();
+      while (!mbar_try_wait(drain, 0) && global_timer_ns() - t0 < 200000000ull) {}
+    }
+  } else {
+    // ---------------------------------------------------------- epilogue --
+    const int q = warp % 4;            // TMEM lane quarter this warp may read
+    const int hf = (warp - 2) / 4;     // which half of the tile's columns
+    const int rl = q * 32 + lane;      // row inside the tile
+    const uint32_t lane_base = (uint32_t)(q * 32) << 16;
+    uint32_t acc_iter = 0, tile_iter = 0;
+    bool ok = true;
+    const int nkb = p.K / 128;
+    for (int item = blockIdx.x; item < total; item += gridDim.x) {
+      const Item it = decode_item(item, p.n_tiles, p.G, s_mt, s_off);
+      const bool shared = (it.g == p.E);
+      const int64_t row = (int64_t)it.row0 + rl;
+      const bool row_ok = rl < it.valid;
+      if (!kFP8) {
+        const uint32_t b = acc_iter & 1u, tph = (acc_iter >> 1) & 1u;
+        if (ok) ok = warp_wait(&tfull[b], tph, p.status, abort_flag);
+        tc_fence_after_sync();
+        const uint32_t base = tmem + lane_base + b * 256;
+        if (kGemm1) {
+          uint16_t* hout = static_cast<uint16_t*>(p.out);
+#pragma unroll
+          for (int ch = 0; ch < 2; ++ch) {
+            uint32_t g[32], u[32];
+            tmem_ld32(base + hf * 64 + ch * 32, g);
+            tmem_ld32(base + 128 + hf * 64 + ch * 32, u);
+            tmem_ld_wait();
+            uint32_t pk[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+              pk[i] = pack_bf16x2(silu_mul(__uint_as_float(g[2 * i]), __uint_as_float(u[2 * i])),
+                                  silu_mul(__uint_as_float(g[2 * i + 1]), __uint_as_float(u[2 * i + 1])));
+            if (ok && row_ok) {
+              uint4* dst = reinterpret_cast<uint4*>(hout + row * p.N + it.n * 128 + hf * 64 + ch * 32);
+#pragma unroll
+              for (int v = 0; v < 4; ++v) dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+            }
+          }
+        } else {
+          uint16_t* yout = static_cast<uint16_t*>(p.out);
+          const float gw = row_ok ? p.row_gate[row] : 0.0f;
+          const int col0 = it.n * 256 + hf * 128;
+#pragma unroll
+          for (int ch = 0; ch < 4; ++ch) {
+            uint32_t v[32];
+            tmem_ld32(base + hf * 128 + ch * 32, v);
+            tmem_ld_wait();
+            uint32_t pk[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+              pk[i] = pack_bf16x2(__uint_as_float(v[2 * i]) * gw, __uint_as_float(v[2 * i + 1]) * gw);
+            if (ok && row_ok && col0 < p.N) {
+              uint4* dst = reinterpret_cast<uint4*>(yout + row * p.N + col0 + ch * 32);
+#pragma unroll
+              for (int w = 0; w < 4; ++w) dst[w] = make_uint4(pk[4 * w], pk[4 * w + 1], pk[4 * w + 2], pk[4 * w + 3]);
+            }
+          }
+        }
+        tc_fence_before_sync();
+        mbar_arrive(&tempty[b]);
+        ++acc_iter;
+      } else {
+        // FP8: promote each K block's partial with its two block scales.
+        float2 acc[64];
+#pragma unroll
+        for (int i = 0; i < 64; ++i) acc[i] = make_float2(0.0f, 0.0f);
+        const float* sa = p.a_scale + row;
+        const float *sb0, *sb1;
+        if (kGemm1) {
+          const int64_t blk = shared ? (int64_t)it.n : ((int64_t)it.g * (p.N / 128) + it.n);
+          sb0 = (shared ? p.bs_scale0 : p.b_scale0) + blk * nkb;
+          sb1 = (shared ? p.bs_scale1 : p.b_scale1) + blk * nkb;
+        } else {
+          const int nb = it.n * 2 + hf;
+          const int64_t blk = shared ? (int64_t)nb : ((int64_t)it.g * (p.N / 128) + nb);
+          sb0 = (shared ? p.bs_scale0 : p.b_scale0) + blk * nkb;
+          sb1 = sb0;
+        }
+        const bool col_ok = kGemm1 || (it.n * 256 + hf * 128 < p.N);
+        for (int kb = 0; kb < nkb; ++kb) {
+          const uint32_t b = acc_iter & 1u, tph = (acc_iter >> 1) & 1u;
+          const float a_s = sa[(int64_t)kb * p.rows_pad];
+          const float f0 = a_s * (col_ok ? sb0[kb] : 0.0f);
+          const float f1 = kGemm1 ? a_s * sb1[kb] : f0;
+          if (ok) ok = warp_wait(&tfull[b], tph, p.status, abort_flag);
+          tc_fence_after_sync();
+          const uint32_t base = tmem + lane_base + b * 256;
+#pragma unroll
+          for (int ch = 0; ch < 4; ++ch) {
+            uint32_t v[32];
+            // GEMM1: chunks 0,1 = gate columns, 2,3 = up columns of this half.
+            const uint32_t col = kGemm1 ? ((ch < 2 ? 0u : 128u) + hf * 64 + (ch & 1) * 32) : (hf * 128 + ch * 32);
+            tmem_ld32(base + col, v);
+            tmem_ld_wait();
+            const float f = (kGemm1 && ch >= 2) ? f1 : f0;
+            const float2 ff = make_float2(f, f);
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+              acc[ch * 16 + i] = fma2(make_float2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1])), ff,
+                                      acc[ch * 16 + i]);
+          }
+          tc_fence_before_sync();
+          mbar_arrive(&tempty[b]);
+          ++acc_iter;
+        }
+        if (kGemm1) {
+          // SwiGLU, then the 1x128 block quantisation of h (the block spans both halves).
+          float hv[64];
+          float amax = 0.0f;
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            hv[2 * i] = silu_mul(acc[i].x, acc[32 + i].x);
+            hv[2 * i + 1] = silu_mul(acc[i].y, acc[32 + i].y);
+            amax = fmaxf(amax, fmaxf(fabsf(hv[2 * i]), fabsf(hv[2 * i + 1])));
+          }
+          float* ax = amax_x + (tile_iter & 1u) * 256;
+          ax[hf * 128 + rl] = amax;
+          named_bar_sync(1, 256);
+          amax = fmaxf(amax, ax[(1 - hf) * 128 + rl]);
+          const float s = amax > 0.0f ? __fdiv_rn(amax, 448.0f) : 1.0f;
+          const float inv = amax > 0.0f ? __frcp_rn(s) : 0.0f;
+          uint32_t pk[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const uint32_t lo = __nv_cvt_float2_to_fp8x2(make_float2(hv[4 * i] * inv, hv[4 * i + 1] * inv),
+                                                         __NV_SATFINITE, __NV_E4M3);
+            const uint32_t hi = __nv_cvt_float2_to_fp8x2(make_float2(hv[4 * i + 2] * inv, hv[4 * i + 3] * inv),
+                                                         __NV_SATFINITE, __NV_E4M3);
+            pk[i] = lo | (hi << 16);
+          }
+          if (ok && row_ok) {
+            uint8_t* hout = static_cast<uint8_t*>(p.out);
+            uint4* dst = reinterpret_cast<uint4*>(hout + row * p.N + it.n * 128 + hf * 64);
+#pragma unroll
+            for (int v = 0; v < 4; ++v) dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+            if (hf == 0) p.out_scale[(int64_t)it.n * p.rows_pad + row] = s;
+          }
+          ++tile_iter;
+        } else {
+          uint16_t* yout = static_cast<uint16_t*>(p.out);
+          const float gw = row_ok ? p.row_gate[row] : 0.0f;
+          if (ok && row_ok && col_ok) {
+            uint4* dst = reinterpret_cast<uint4*>(yout + row * p.N + it.n * 256 + hf * 128);
+#pragma unroll
+            for (int w = 0; w < 16; ++w) {
+              const float2 a0 = acc[4 * w], a1 = acc[4 * w + 1], a2 = acc[4 * w + 2], a3 = acc[4 * w + 3];
+              dst[w] = make_uint4(pack_bf16x2(a0.x * gw, a0.y * gw), pack_bf16x2(a1.x * gw, a1.y * gw),
+                                  pack_bf16x2(a2.x * gw, a2.y * gw), pack_bf16x2(a3.x * gw, a3.y * gw));
+            }
+          }
+        }
+      }
+    }
+  }
+  tc_fence_before_sync();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after_sync();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+template <bool kFP8, bool kGemm1>
+cudaError_t launch_one(const GemmParams& p, int grid, const CUtensorMap& a, const CUtensorMap& b0,
+                       const CUtensorMap& b1, const CUtensorMap& bs0, const CUtensorMap& bs1, cudaStream_t s) {
+  auto kern = grouped_gemm_kernel<kFP8, kGemm1>;
+  cudaError_t e =
+      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SmemLayout::kDynamic);
+  if (e != cudaSuccess) return e;
+  kern<<<grid, kThreads, SmemLayout::kDynamic, s>>>(p, a, b0, b1, bs0, bs1);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_gemm1(const GemmParams& p, bool fp8, int grid, const CUtensorMap& tm_a, const CUtensorMap& tm_w1,
+                         const CUtensorMap& tm_w3, const CUtensorMap& tm_sw1, const CUtensorMap& tm_sw3,
+                         cudaStream_t s) {
+  return fp8 ? launch_one<true, true>(p, grid, tm_a, tm_w1, tm_w3, tm_sw1, tm_sw3, s)
+             : launch_one<false, true>(p, grid, tm_a, tm_w1, tm_w3, tm_sw1, tm_sw3, s);
+}
+
+cudaError_t launch_gemm2(const GemmParams& p, bool fp8, int grid, const CUtensorMap& tm_a, const CUtensorMap& tm_w2,
+                         const CUtensorMap& tm_sw2, cudaStream_t s) {
+  return fp8 ? launch_one<true, false>(p, grid, tm_a, tm_w2, tm_w2, tm_sw2, tm_sw2, s)
+             : launch_one<false, false>(p, grid, tm_a, tm_w2, tm_w2, tm_sw2, tm_sw2, s);
+}
+
+}  // namespace moe

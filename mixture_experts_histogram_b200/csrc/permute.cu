@@ -1,0 +1,196 @@
+// Token -> expert histogram, its exclusive scan, and the gather indices (the
+// "critical MoE primitives" of the StepFun "Step-5 minimal inference" README,
+// opening section). Groups 0..E-1 are the routed experts; group E is the
+// shared expert, which takes every token (NeMo "Step-5-Preview" page: one
+// shared expert, here treated as one more group of the grouped GEMMs).
+//
+// Row order is fixed and independent of scheduling: groups in index order,
+// and inside a group the tokens ascend. Atomics only count; they never decide
+// where a row goes:
+//   1. histogram: one CTA per 256-token chunk counts its (token, slot) pairs
+//      per expert in shared memory -> chunk_base[e][chunk].
+//   2. scan: one CTA scans chunk counts per expert (one warp per expert), then
+//      the expert totals -> counts, offsets, and the per-group M-tile prefix
+//      the grouped GEMMs schedule from; chunk_base becomes absolute row bases.
+//   3. scatter: each warp ranks its 32 tokens' pairs in (token, slot) order
+//      with __match_any_sync (equal experts in one 32-pair round rank by lane),
+//      warps are then offset by an exclusive scan over the CTA's 8 warps, and
+//      rows are written: perm[row] = token, pos[token, slot] = row,
+//      row_gate[row] = gate.
+#include "common.cuh"
+#include "ptx.cuh"
+
+namespace moe {
+
+namespace {
+
+__global__ void __launch_bounds__(256) histogram_kernel(const PermuteParams p) {
+  __shared__ int cnt[kMaxExperts];
+  for (int e = threadIdx.x; e < p.E; e += blockDim.x) cnt[e] = 0;
+  __syncthreads();
+  const int64_t t0 = (int64_t)blockIdx.x * kHistChunk;
+  const int64_t ntok = min((int64_t)kHistChunk, (int64_t)p.T - t0);
+  const int64_t npairs = ntok * p.k;
+  const int32_t* idx = p.idx + t0 * p.k;
+  for (int64_t i = threadIdx.x; i < npairs; i += blockDim.x) {
+    const int e = idx[i];
+    if (e < 0 || e >= p.E) latch_status(p.status, MOE_ERR_BAD_INDEX);
+    else atomicAdd(&cnt[e], 1);
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < p.E; e += blockDim.x) p.chunk_base[(int64_t)e * p.chunks + blockIdx.x] = cnt[e];
+}
+
+__device__ __forceinline__ int warp_inclusive_scan(int v, int lane) {
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int o = __shfl_up_sync(0xffffffffu, v, off);
+    if (lane >= off) v += o;
+  }
+  return v;
+}
+
+__global__ void __launch_bounds__(1024) scan_kernel(const PermuteParams p) {
+  __shared__ int cnt_s[kMaxExperts + 1];
+  __shared__ int off_s[kMaxExperts + 2];
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  // per-expert exclusive scan over chunks (bases relative to the expert)
+  for (int e = warp; e < p.E; e += 32) {
+    int running = 0;
+    int32_t* row = p.chunk_base + (int64_t)e * p.chunks;
+    for (int c0 = 0; c0 < p.chunks; c0 += 32) {
+      const int c = c0 + lane;
+      const int v = c < p.chunks ? row[c] : 0;
+      const int incl = warp_inclusive_scan(v, lane);
+      if (c < p.chunks) row[c] = running + incl - v;
+      running += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    if (lane == 0) cnt_s[e] = running;
+  }
+  if (threadIdx.x == 0 && p.S) cnt_s[p.E] = p.T;
+  __syncthreads();
+  // offsets and M-tile prefix over the G groups
+  if (warp == 0) {
+    int run_off = 0, run_mt = 0;
+    for (int g0 = 0; g0 < p.G; g0 += 32) {
+      const int g = g0 + lane;
+      const int c = g < p.G ? cnt_s[g] : 0;
+      const int mt = (c + kTileM - 1) / kTileM;
+      const int ic = warp_inclusive_scan(c, lane);
+      const int im = warp_inclusive_scan(mt, lane);
+      if (g < p.G) {
+        p.counts[g] = c;
+        p.offsets[g] = run_off + ic - c;
+        p.mt_prefix[g] = run_mt + im - mt;
+        off_s[g] = run_off + ic - c;
+      }
+      run_off += __shfl_sync(0xffffffffu, ic, 31);
+      run_mt += __shfl_sync(0xffffffffu, im, 31);
+    }
+    if (lane == 0) {
+      p.offsets[p.G] = run_off;
+      p.mt_prefix[p.G] = run_mt;
+    }
+  }
+  __syncthreads();
+  const int64_t n = (int64_t)p.E * p.chunks;
+  for (int64_t i = threadIdx.x; i < n; i += blockDim.x) p.chunk_base[i] += off_s[i / p.chunks];
+}
+
+__global__ void __launch_bounds__(256) scatter_kernel(const PermuteParams p) {
+  __shared__ int wcnt[8][kMaxExperts];
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  for (int i = threadIdx.x; i < 8 * kMaxExperts; i += blockDim.x) (&wcnt[0][0])[i] = 0;
+  __syncthreads();
+
+  const int64_t tw0 = (int64_t)blockIdx.x * kHistChunk + warp * 32;  // this warp's first token
+  int rank[kMaxTopK];
+  int ekeep[kMaxTopK];
+  // Pass 1: ranks inside the warp, pairs taken in (token, slot) order, 32 per round.
+#pragma unroll
+  for (int r = 0; r < kMaxTopK; ++r) {
+    ekeep[r] = -1;
+    rank[r] = 0;
+    if (r < p.k) {
+      const int pidx = r * 32 + lane;
+      const int64_t t = tw0 + pidx / p.k;
+      const int j = pidx % p.k;
+      int e = -1;
+      if (t < p.T) {
+        e = p.idx[t * p.k + j];
+        if (e < 0 || e >= p.E) e = -1;
+      }
+      const int key = e >= 0 ? e : (0x40000000 + lane);  // unmatched sentinel for empty lanes
+      const unsigned m = __match_any_sync(0xffffffffu, key);
+      const int rk = __popc(m & ((1u << lane) - 1u));
+      const int prev = e >= 0 ? wcnt[warp][e] : 0;
+      __syncwarp();
+      if (e >= 0 && rk == 0) wcnt[warp][e] = prev + __popc(m);
+      __syncwarp();
+      rank[r] = prev + rk;
+      ekeep[r] = e;
+    }
+  }
+  __syncthreads();
+  // Pass 2: warp offsets per expert, on top of this chunk's absolute base.
+  for (int e = threadIdx.x; e < p.E; e += blockDim.x) {
+    int run = p.chunk_base[(int64_t)e * p.chunks + blockIdx.x];
+#pragma unroll
+    for (int w = 0; w < 8; ++w) {
+      const int v = wcnt[w][e];
+      wcnt[w][e] = run;
+      run += v;
+    }
+  }
+  __syncthreads();
+  // Pass 3: write the rows.
+  const int S = p.S + p.k;
+#pragma unroll
+  for (int r = 0; r < kMaxTopK; ++r) {
+    if (r < p.k) {
+      const int pidx = r * 32 + lane;
+      const int64_t t = tw0 + pidx / p.k;
+      const int j = pidx % p.k;
+      if (t < p.T) {
+        const int e = ekeep[r];
+        if (e >= 0) {
+          const int row = wcnt[warp][e] + rank[r];
+          p.perm[row] = (int32_t)t;
+          p.pos[t * S + j] = row;
+          if (p.row_gate) p.row_gate[row] = p.gate[t * p.k + j];
+        } else {
+          p.pos[t * S + j] = -1;  // a skipped (bad-index) pair
+        }
+      }
+    }
+  }
+  // The shared expert's rows: token order.
+  if (p.S) {
+    const int64_t t = (int64_t)blockIdx.x * kHistChunk + threadIdx.x;
+    if (t < p.T) {
+      const int row = p.offsets[p.E] + (int)t;
+      p.perm[row] = (int32_t)t;
+      p.pos[t * S + p.k] = row;
+      if (p.row_gate) p.row_gate[row] = 1.0f;
+    }
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_histogram(const PermuteParams& p, cudaStream_t s) {
+  histogram_kernel<<<p.chunks, 256, 0, s>>>(p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_scan(const PermuteParams& p, cudaStream_t s) {
+  scan_kernel<<<1, 1024, 0, s>>>(p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_scatter(const PermuteParams& p, cudaStream_t s) {
+  scatter_kernel<<<p.chunks, 256, 0, s>>>(p);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

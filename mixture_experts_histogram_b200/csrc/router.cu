@@ -1,0 +1,226 @@
+// Router: fp32 logits l = x . Wr^T on the tensor cores, then per token the
+// top-k selection (ties to the lower expert index) and the softmax gates
+// renormalised over the chosen k.
+//
+// Layer definition: NeMo AutoModel "Step-5-Preview" page, "Model Architecture"
+// table (352 routed experts, top-8 routing, a learned router).
+//
+// Logits GEMM: one CTA per (128-token tile, K split). Warp 0 streams x and Wr
+// tiles with TMA into a 3-4 stage ring of 128B-swizzled shared-memory tiles;
+// warp 1 issues tcgen05 MMAs (M = 128 tokens, N = up to 2 x 256 experts) into a
+// TMEM accumulator; warps 2-5 read the accumulator back (one token row per
+// thread) and store fp32 partial logits. Small T is split along K so that the
+// 2.9 MB of router weights are streamed by many SMs at once; the top-k kernel
+// adds the K-split partials in a fixed order.
+#include <cuda_bf16.h>
+#include <math.h>
+
+#include "common.cuh"
+#include "ptx.cuh"
+
+namespace moe {
+
+namespace {
+
+constexpr int kRouterThreads = 192;
+constexpr int kRouterMaxStages = 4;
+constexpr int kASmem = kTileM * kStageBytesK;  // 16 KB of x per stage
+
+__host__ __device__ inline int router_b_bytes(const RouterParams& p) { return p.nbox * p.box_rows * kStageBytesK; }
+
+__host__ __device__ inline int router_stages(const RouterParams& p) {
+  const int per = kASmem + router_b_bytes(p);
+  int st = (200 * 1024) / per;
+  return st > kRouterMaxStages ? kRouterMaxStages : st;
+}
+
+__global__ void __launch_bounds__(kRouterThreads, 1)
+    router_gemm_kernel(const RouterParams p, const __grid_constant__ CUtensorMap tm_x,
+                       const __grid_constant__ CUtensorMap tm_w) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int stages = router_stages(p);
+  const int bbytes = router_b_bytes(p);
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + stages * kASmem;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sB + stages * bbytes);
+  uint64_t* empty = full + kRouterMaxStages;
+  uint64_t* done = empty + kRouterMaxStages;
+  uint64_t* drain = done + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int m_tile = blockIdx.x, split = blockIdx.y;
+  const int ks0 = (int)((int64_t)split * p.kstages / p.ksplit);
+  const int ks1 = (int)((int64_t)(split + 1) * p.kstages / p.ksplit);
+  const int ncols = p.nbox * p.box_rows;
+  const uint32_t tmem_cols = ncols <= 32 ? 32 : ncols <= 64 ? 64 : ncols <= 128 ? 128 : ncols <= 256 ? 256 : 512;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < stages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(done, 1);
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tm_x);
+    tma_prefetch_desc(&tm_w);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, tmem_cols);
+    tmem_relinquish();
+  }
+  __syncthreads();
+  tc_fence_after_sync();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0 && lane == 0) {
+    // ---- TMA producer ----
+    int stage = 0;
+    uint32_t phase = 0;
+    for (int ks = ks0; ks < ks1; ++ks) {
+      if (!mbar_wait(&empty[stage], phase ^ 1, p.status, abort_flag)) break;
+      mbar_arrive_expect_tx(&full[stage], kASmem + bbytes);
+      tma_load_2d(sA + stage * kASmem, &tm_x, &full[stage], ks * 64, m_tile * kTileM);
+      for (int b = 0; b < p.nbox; ++b)
+        tma_load_2d(sB + stage * bbytes + b * p.box_rows * kStageBytesK, &tm_w, &full[stage], ks * 64,
+                    b * p.box_rows);
+      if (++stage == stages) { stage = 0; phase ^= 1; }
+    }
+  } else if (warp == 1 && lane == 0) {
+    // ---- MMA issuer ----
+    const uint32_t idesc = idesc_mma(1, kTileM, p.box_rows);
+    int stage = 0;
+    uint32_t phase = 0;
+    bool ok = true;
+    for (int ks = ks0; ks < ks1; ++ks) {
+      if (!mbar_wait(&full[stage], phase, p.status, abort_flag)) { ok = false; break; }
+      tc_fence_after_sync();
+      const uint64_t adesc = sdesc_k_sw128(sA + stage * kASmem);
+      for (int kk = 0; kk < 4; ++kk) {
+        for (int b = 0; b < p.nbox; ++b) {
+          const uint64_t bdesc = sdesc_k_sw128(sB + stage * bbytes + b * p.box_rows * kStageBytesK);
+          mma_bf16(tmem + b * p.box_rows, adesc + 2 * kk, bdesc + 2 * kk, idesc, (ks > ks0 || kk > 0) ? 1u : 0u);
+        }
+      }
+      mma_commit(&empty[stage]);
+      if (++stage == stages) { stage = 0; phase ^= 1; }
+    }
+    if (ok) mma_commit(done);
+    // Drain: every MMA issued so far has completed once this arrives.
+    mma_commit(drain);
+    mbar_wait(drain, 0, p.status, abort_flag);
+  } else if (warp >= 2) {
+    // ---- epilogue: one token row per thread ----
+    const int q = warp % 4;
+    const int row = m_tile * kTileM + q * 32 + lane;
+    bool ok = mbar_wait(done, 0, p.status, abort_flag);
+    ok = __all_sync(0xffffffffu, ok);
+    if (ok) {
+      tc_fence_after_sync();
+      float* dst = p.partial + ((int64_t)split * p.T + row) * p.E;
+      for (int c0 = 0; c0 < ncols; c0 += 32) {
+        uint32_t v[32];
+        tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)c0, v);
+        tmem_ld_wait();
+        if (row < p.T) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i)
+            if (c0 + i < p.E) dst[c0 + i] = __uint_as_float(v[i]);
+        }
+      }
+    }
+  }
+  tc_fence_before_sync();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after_sync();
+    tmem_dealloc(tmem, tmem_cols);
+  }
+}
+
+// One warp per token: sum the K-split partial logits in split order, add the
+// bias, pick the top k (largest logit first, ties to the lower index), and
+// renormalise their softmax probabilities.
+__global__ void __launch_bounds__(256) topk_kernel(const TopkParams p) {
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int64_t t = (int64_t)blockIdx.x * 8 + warp;
+  if (t >= p.T) return;
+  constexpr int kPer = kMaxExperts / 32;
+  float l[kPer];
+#pragma unroll
+  for (int i = 0; i < kPer; ++i) {
+    const int e = lane + 32 * i;
+    float v = -INFINITY;
+    if (e < p.E) {
+      v = 0.0f;
+      for (int s = 0; s < p.ksplit; ++s) v += p.partial[((int64_t)s * p.T + t) * p.E + e];
+      if (p.bias) v += p.bias[e];
+      if (p.logits) p.logits[t * p.E + e] = v;
+    }
+    l[i] = v;
+  }
+  uint32_t taken = 0;
+  float my_v = -INFINITY;
+  int my_e = 0;
+  for (int j = 0; j < p.k; ++j) {
+    float bv = -INFINITY;
+    int be = 0x7FFFFFFF;
+#pragma unroll
+    for (int i = 0; i < kPer; ++i) {
+      const int e = lane + 32 * i;
+      if (e < p.E && !(taken & (1u << i)) && (l[i] > bv || (l[i] == bv && e < be))) {
+        bv = l[i];
+        be = e;
+      }
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+      const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
+      const int oe = __shfl_xor_sync(0xffffffffu, be, off);
+      if (ov > bv || (ov == bv && oe < be)) {
+        bv = ov;
+        be = oe;
+      }
+    }
+    if ((be & 31) == lane) taken |= 1u << (be >> 5);
+    if (lane == j) {
+      my_v = bv;
+      my_e = be;
+    }
+  }
+  const float m = __shfl_sync(0xffffffffu, my_v, 0);
+  const float w = (lane < p.k) ? expf(my_v - m) : 0.0f;
+  float z = w;
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) z += __shfl_xor_sync(0xffffffffu, z, off);
+  if (lane < p.k) {
+    p.idx[t * p.k + lane] = my_e;
+    p.gate[t * p.k + lane] = w / z;
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_router_gemm(const RouterParams& p, const CUtensorMap& tm_x, const CUtensorMap& tm_w,
+                               cudaStream_t s) {
+  const int stages = router_stages(p);
+  const size_t smem = 1024 + (size_t)stages * (kASmem + router_b_bytes(p)) + 256;
+  cudaError_t e = cudaFuncSetAttribute(router_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  dim3 grid((unsigned)ceil_div(p.T, kTileM), (unsigned)p.ksplit);
+  router_gemm_kernel<<<grid, kRouterThreads, smem, s>>>(p, tm_x, tm_w);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_topk(const TopkParams& p, cudaStream_t s) {
+  topk_kernel<<<(unsigned)ceil_div(p.T, 8), 256, 0, s>>>(p);
+  return cudaGetLastError();
+}
+
+}  // namespace moe
