@@ -1,0 +1,406 @@
+#!/usr/bin/env python
+"""Benchmark of the Step-5 routed-MoE layer forward on B200. Prints one JSON line.
+
+Headline workload: the Step-5 MoE layer prefill with FP8 experts, T = 8192
+tokens (hidden 4096, 352 routed experts, top-8, one shared expert,
+intermediate 1536; 128x128 E4M3 weight blocks, 1x128 E4M3 activations).
+A step is one whole layer forward (router, top-k, histogram/scan/permute,
+gather+quantise, gate/up GEMM + SwiGLU, down GEMM, combine) through the C ABI
+on inputs already resident in HBM. The line also carries the FP8 decode
+workload (T = 64) that the metric quotes, measured the same way.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+N > 1 runs N independent replicas (one per GPU; the layer does not shard on
+one node in this design) under torchrun; the value is the tokens of all ranks
+over the slowest rank's time. --impl reference times the CPU oracle instead.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "Step-5 MoE layer tokens/s (FP8, T=8192 / T=64) and % of FP8 / HBM roofline"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
+L2_FLUSH_BYTES = 256 << 20
+KERNELS = ["router_gemm", "router_topk", "histogram", "scan", "scatter", "gather", "gemm1_gate_up_swiglu",
+           "gemm2_down", "combine"]
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=["prefill-fp8", "decode-bf16", "long-skew-fp8"], default="prefill-fp8")
+    ap.add_argument("--no-decode", action="store_true", help="skip the T=64 FP8 decode line")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--tokens", type=int, default=None, help="override T (profiling cases)")
+    ap.add_argument("--experts", type=int, default=None, help="override E (profiling cases)")
+    return ap.parse_args()
+
+
+def workload(name, tokens=None, experts=None):
+    import dataclasses
+    import synth
+    s = {"prefill-fp8": synth.PREFILL_FP8, "decode-bf16": synth.DECODE_BF16,
+         "long-skew-fp8": synth.LONG_SKEW_FP8}[name]
+    if experts is not None:
+        s = dataclasses.replace(s, n_experts=experts, name=f"{s.name}-E{experts}")
+    if tokens is not None:
+        s = s.with_tokens(tokens)
+    return s
+
+
+def describe(shape) -> dict:
+    return {"workload": f"{shape.name}: T={shape.T} H={shape.hidden} E={shape.n_experts} top-{shape.top_k} "
+                        f"shared={shape.n_shared} I={shape.inter} "
+                        f"{'FP8 E4M3 128x128 weights, 1x128 activations' if shape.wdtype else 'BF16'}"
+                        f"{', Zipf-skewed routing' if shape.skew else ', uniform routing'}",
+            "tokens": shape.T, "hidden": shape.hidden, "experts": shape.n_experts, "top_k": shape.top_k,
+            "shared_experts": shape.n_shared, "inter": shape.inter, "seed": shape.seed,
+            "l2": "flushed between timed steps (256 MB write)"}
+
+
+def peaks():
+    p = dict(FALLBACK_PEAKS)
+    src = "fallback"
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        try:
+            d = json.load(open(path))
+            p["hbm_gbs"] = float(d["hbm_gbs"])
+            p["bf16_tflops"] = float(d["bf16_tflops"])
+            src = "measured"
+        except Exception:
+            pass
+    p["fp8_tflops"] = 2.0 * p["bf16_tflops"]  # nominal FP8:BF16 dense ratio 2
+    p["source"] = src
+    return p
+
+
+# ------------------------------------------------------------------ clocks --
+
+class ClockSampler:
+    """nvidia-smi clock/throttle sampling while the timed region runs."""
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_{os.getpid()}.csv")
+
+    def __enter__(self):
+        os.makedirs(os.path.dirname(self.path), exist_ok=True)
+        q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+        try:
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={q}", "--format=csv,noheader,nounits",
+                                          "-i", str(self.gpu), "-lms", "100"], stdout=self.fh,
+                                         stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            time.sleep(0.2)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+            self.fh.close()
+
+    def summary(self):
+        if self.proc is None or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["clock sampling unavailable"]}
+        sm, mx, reasons, power = [], None, set(), []
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+                power.append(float(f[3]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        loaded = [s for s, p in zip(sm, power) if p > 250.0] or sm
+        return {"sm_mhz": statistics.median(loaded) if loaded else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm), "samples_under_load": len(loaded)}
+
+
+# --------------------------------------------------------------- our arm ----
+
+def run_ours(args):
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+    import synth
+    import mixture_experts_histogram_b200 as m
+    from mixture_experts_histogram_b200 import build as mbuild
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    if rank == 0:
+        mbuild.build()
+    if world > 1:
+        dist.barrier()
+    m.load()
+    shape = workload(args.workload, args.tokens, args.experts)
+    x_np = synth.make_x(shape)
+    w_np = synth.make_weights(shape)
+    wd = m.upload_weights(w_np, f"cuda:{local}")
+    wts = m.make_weights(wd)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=f"cuda:{local}")
+    stream = torch.cuda.current_stream()
+
+    def measure(T, x_host, e2e=True, profile=True):
+        cfg = m.make_config(shape.hidden, shape.n_experts, shape.top_k, shape.n_shared, shape.inter, shape.wdtype)
+        x = m.to_device(x_host, f"cuda:{local}")
+        out = torch.empty((T, shape.hidden), dtype=torch.bfloat16, device=f"cuda:{local}")
+        idx = torch.empty((T, shape.top_k), dtype=torch.int32, device=f"cuda:{local}")
+        gate = torch.empty((T, shape.top_k), dtype=torch.float32, device=f"cuda:{local}")
+        ws = torch.empty(m.moe_workspace_bytes(cfg, T), dtype=torch.uint8, device=f"cuda:{local}")
+
+        def step():
+            m.moe_forward(cfg, T, x, wts, out, ws, topk_idx=idx, topk_w=gate, stream=stream)
+
+        for _ in range(args.warmup):
+            flush.fill_(1)
+            step()
+        st = m.moe_read_status(ws)
+        if st != 0:
+            raise RuntimeError(f"device status after warm-up: {m.moe_status_string(st)}")
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+        per_kernel = {k: 0.0 for k in KERNELS}
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        m.moe_profile_enable(profile)
+        for i in range(args.steps):
+            flush.fill_(i & 0xFF)
+            torch.cuda._sleep(200000)  # ~0.1 ms of GPU time so the host has queued the step before ev0
+            ev[i][0].record(stream)
+            step()
+            ev[i][1].record(stream)
+            if profile:
+                for k, v in m.moe_profile_read().items():
+                    per_kernel[k] += v
+        torch.cuda.synchronize()
+        m.moe_profile_enable(False)
+        if world > 1:
+            dist.barrier()
+        total_ms = sum(a.elapsed_time(b) for a, b in ev)
+        t = torch.tensor([total_ms], dtype=torch.float64, device=f"cuda:{local}")
+        if world > 1:
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+        st = m.moe_read_status(ws)
+        if st != 0:
+            raise RuntimeError(f"device status after timing: {m.moe_status_string(st)}")
+        res = {"ms_per_step": total_ms / args.steps, "tokens_per_s": world * T * args.steps / (total_ms / 1e3),
+               "kernel_ms": {k: v / args.steps for k, v in per_kernel.items()},
+               "idx": idx.cpu().numpy()}
+        if e2e:
+            xh = torch.from_numpy(np.ascontiguousarray(x_host).view(np.int16)).pin_memory()
+            oh = torch.empty((T, shape.hidden), dtype=torch.int16).pin_memory()
+            for _ in range(2):
+                m.moe_forward_host(cfg, T, xh, wts, oh, ws, stream=stream)
+            ms = []
+            for i in range(args.steps):
+                flush.fill_(i & 0xFF)
+                torch.cuda.synchronize()
+                t0 = time.perf_counter()
+                m.moe_forward_host(cfg, T, xh, wts, oh, ws, stream=stream)
+                ms.append((time.perf_counter() - t0) * 1e3)
+            tt = torch.tensor([sum(ms)], dtype=torch.float64, device=f"cuda:{local}")
+            if world > 1:
+                dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+            res["e2e"] = {"value": world * T * args.steps / (float(tt.item()) / 1e3), "unit": "tokens/s",
+                          "h2d_bytes_per_step": T * shape.hidden * 2, "d2h_bytes_per_step": T * shape.hidden * 2}
+        return res
+
+    pk = peaks()
+    with ClockSampler(local) as clk:
+        main = measure(shape.T, x_np, e2e=not args.no_e2e)
+        decode = None
+        if not args.no_decode and shape.wdtype == synth.WDTYPE_FP8 and shape.T != 64:
+            dshape = shape.with_tokens(64)
+            decode = measure(64, synth.make_x(dshape), e2e=False)
+    clocks = clk.summary()
+
+    def roofline(res, T):
+        """The dominant kernel against its bound (HBM bytes or tensor FLOPs)."""
+        idx = res["idx"]
+        touched = int(np.unique(idx).size)
+        es = 1 if shape.wdtype else 2
+        H, I, E, k, S = shape.hidden, shape.inter, shape.n_experts, shape.top_k, shape.n_shared
+        R = (k + S) * T
+        groups = touched + S
+        scale1 = (2 * (I // 128) * (H // 128) * 4) if shape.wdtype else 0
+        scale2 = ((H // 128) * (I // 128) * 4) if shape.wdtype else 0
+        kern = {
+            "gemm1_gate_up_swiglu": {
+                "bytes": groups * (2 * I * H * es + scale1) + T * H * es + R * I * es,
+                "flops": 2.0 * R * H * 2 * I},
+            "gemm2_down": {"bytes": groups * (H * I * es + scale2) + R * I * es + R * H * 2,
+                           "flops": 2.0 * R * I * H},
+        }
+        dom = max(kern, key=lambda kk: res["kernel_ms"].get(kk, 0.0))
+        ms = res["kernel_ms"][dom]
+        t_hbm = kern[dom]["bytes"] / (pk["hbm_gbs"] * 1e9)
+        peak_tf = pk["fp8_tflops"] if shape.wdtype else pk["bf16_tflops"]
+        t_tc = kern[dom]["flops"] / (peak_tf * 1e12)
+        traffic = traffic_for(dom, shape.name if T == shape.T else f"{shape.name}@T={T}")
+        if t_hbm >= t_tc:
+            ach = kern[dom]["bytes"] / (ms / 1e3) / 1e9
+            r = {"bound": "hbm", "achieved": round(ach, 1), "peak": pk["hbm_gbs"], "unit": "GB/s"}
+        else:
+            ach = kern[dom]["flops"] / (ms / 1e3) / 1e12
+            r = {"bound": "tensor", "achieved": round(ach, 1), "peak": peak_tf, "unit": "TFLOP/s"}
+        r.update({"frac": round(ach / r["peak"], 4), "traffic": traffic, "kernel": dom,
+                  "kernel_ms": round(ms, 4), "algorithmic_bytes": kern[dom]["bytes"],
+                  "algorithmic_flops": kern[dom]["flops"], "touched_experts": touched,
+                  "peak_source": f"{pk['source']} (MEASURED_PEAKS.json; FP8 = 2 x measured BF16)"})
+        # Whole layer against max(compute, bytes): weights of touched experts + router + x + out.
+        lay_bytes = (groups * (3 * I * H * es + scale1 + scale2) + E * H * 2 + 2 * T * H * 2)
+        lay_flops = 2.0 * T * H * E + 2.0 * 3 * H * I * R
+        t_roof = max(lay_bytes / (pk["hbm_gbs"] * 1e9), lay_flops / (peak_tf * 1e12))
+        layer = {"ms": round(res["ms_per_step"], 4), "roofline_ms": round(t_roof * 1e3, 4),
+                 "frac": round(t_roof * 1e3 / res["ms_per_step"], 4),
+                 "tflops": round(lay_flops / (res["ms_per_step"] / 1e3) / 1e12, 1),
+                 "hbm_gbs_of_algorithmic_bytes": round(lay_bytes / (res["ms_per_step"] / 1e3) / 1e9, 1)}
+        return r, layer
+
+    roof, layer = roofline(main, shape.T)
+    line = {
+        "metric": METRIC, "value": round(main["tokens_per_s"], 1), "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(main["ms_per_step"], 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "e4m3" if shape.wdtype else "bf16", "data": "synthetic (seeded, counter-based generator)",
+        "config": dict(describe(shape), parallelism=f"replicas x{world}" if world > 1 else "single GPU"),
+        "roofline": roof, "layer_roofline": layer,
+        "kernel_ms": {k: round(v, 4) for k, v in main["kernel_ms"].items()},
+        "e2e": main.get("e2e"), "gpu_launches": len(KERNELS) * args.steps, "clocks": clocks,
+    }
+    if decode is not None:
+        droof, dlayer = roofline(decode, 64)
+        line["decode_t64"] = {"value": round(decode["tokens_per_s"], 1), "unit": "tokens/s",
+                              "ms_per_step": round(decode["ms_per_step"], 4), "roofline": droof,
+                              "layer_roofline": dlayer,
+                              "kernel_ms": {k: round(v, 4) for k, v in decode["kernel_ms"].items()},
+                              "config": "T=64, same layer and weights as the headline workload"}
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(shape, x_np, w_np)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def traffic_for(kernel: str, workload_name: str):
+    """DRAM bytes per launch from a committed ncu summary, if it matches the current kernel source."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    try:
+        d = json.load(open(path))
+        ent = d.get(kernel, {}).get(workload_name)
+        if not ent or ent.get("source_sha") != kernel_source_sha():
+            return None
+        return ent["dram_bytes_per_launch"]
+    except Exception:
+        return None
+
+
+def kernel_source_sha() -> str:
+    import hashlib
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "mixture_experts_histogram_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        h.update(open(os.path.join(csrc, f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+# --------------------------------------------------------- CPU oracle arm ----
+
+def _oracle_sample(shape, x_np, w_np, n_tok):
+    import oracle
+    t0 = time.perf_counter()
+    xs = x_np[:n_tok]
+    idx, gate, _ = oracle.route(xs, w_np["router_w"], w_np["router_bias"], shape.top_k)
+    oracle.moe_tokens(shape.with_tokens(n_tok), w_np, xs, idx, gate)
+    return time.perf_counter() - t0
+
+
+def _pick_sample(shape, x_np, w_np, target_s):
+    t1 = _oracle_sample(shape, x_np, w_np, 2)
+    per_tok = max(t1 / 2, 1e-4)
+    return int(min(max(2, target_s / per_tok), 512, shape.T))
+
+
+def cpu_baseline(shape, x_np, w_np, target_s=12.0):
+    """The oracle, as it stands, on all host cores, on a bounded token sample."""
+    n = _pick_sample(shape, x_np, w_np, target_s)
+    dt = _oracle_sample(shape, x_np, w_np, n)
+    return {"value": round(n / dt, 3), "unit": "tokens/s", "cores": os.cpu_count(), "kind": "oracle",
+            "sample": f"first {n} tokens of the workload: routing, experts and combine ({dt:.1f} s)"}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import synth
+    shape = workload(args.workload, args.tokens, args.experts)
+    x_np = synth.make_x(shape)
+    w_np = synth.make_weights(shape)
+    steps, warm = args.steps, args.warmup
+    budget = 150.0
+    n = _pick_sample(shape, x_np, w_np, budget / max(1, steps + warm))
+    for _ in range(min(warm, 1)):
+        _oracle_sample(shape, x_np, w_np, n)
+    ts = [_oracle_sample(shape, x_np, w_np, n) for _ in range(steps)]
+    value = n * steps / sum(ts)
+    line = {"metric": METRIC, "value": round(value, 3), "unit": "tokens/s", "n_gpus": 0, "steps": steps,
+            "warmup": warm, "ms_per_step": round(1e3 * sum(ts) / steps, 2), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64 accumulation (oracle)",
+            "data": "synthetic (seeded, counter-based generator)", "impl": "reference",
+            "config": describe(shape),
+            "cpu_baseline": {"value": round(value, 3), "unit": "tokens/s", "cores": os.cpu_count(),
+                             "kind": "oracle", "sample": f"first {n} tokens of the workload per step"},
+            "e2e": {"value": round(value, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    a = parse_args()
+    if a.impl == "reference":
+        run_reference(a)
+    else:
+        run_ours(a)

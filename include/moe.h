@@ -36,7 +36,7 @@
  *    a timed-out wait) are latched in a status word inside the workspace and
  *    read with moe_read_status.
  *  - Device buffers must be 16-byte aligned (TMA); 256-byte alignment is
- *    recommended. The workspace must be 1024-byte aligned.
+ *    recommended. The workspace must be 256-byte aligned.
  *  - Supported shapes: H and I multiples of 128; 1 <= E <= 512;
  *    1 <= top_k <= min(E, 16); n_shared in {0, 1}; 0 <= T, (top_k+n_shared)*T < 2^31.
  *    T == 0 is a no-op that returns MOE_OK.
@@ -75,7 +75,7 @@ enum {
   MOE_ERR_CUDA = 4,               /* a CUDA runtime call failed (no device, launch error, ...) */
   MOE_ERR_BAD_INDEX = 5,          /* device: an expert index outside [0, E) was skipped */
   MOE_ERR_DEVICE_TIMEOUT = 6,     /* device: a bounded wait gave up; results are invalid */
-  MOE_ERR_MISALIGNED = 7          /* a buffer is not 16-byte (workspace: 1024-byte) aligned */
+  MOE_ERR_MISALIGNED = 7          /* a buffer is not 16-byte (workspace: 256-byte) aligned */
 };
 
 typedef struct moe_config {

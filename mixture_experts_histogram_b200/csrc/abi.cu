@@ -300,7 +300,7 @@ int run_combine(const moe_config* c, int64_t T, const void* y, const int32_t* po
 
 int check_ws(const moe_config* c, int64_t T, void* ws, size_t ws_bytes, WsLayout* L) {
   if (!ws) return MOE_ERR_INVALID_ARG;
-  if (!aligned(ws, 1024)) return MOE_ERR_MISALIGNED;
+  if (!aligned(ws, 256)) return MOE_ERR_MISALIGNED;
   *L = ws_layout(*c, T, kRouterTargetCtas);
   if (ws_bytes < L->total) return MOE_ERR_WORKSPACE_TOO_SMALL;
   return MOE_OK;

@@ -409,9 +409,13 @@ template <bool kFP8, bool kGemm1>
 cudaError_t launch_one(const GemmParams& p, int grid, const CUtensorMap& a, const CUtensorMap& b0,
                        const CUtensorMap& b1, const CUtensorMap& bs0, const CUtensorMap& bs1, cudaStream_t s) {
   auto kern = grouped_gemm_kernel<kFP8, kGemm1>;
-  cudaError_t e =
-      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SmemLayout::kDynamic);
-  if (e != cudaSuccess) return e;
+  static bool attr_set = false;  // per process; one device's limit serves every B200
+  if (!attr_set) {
+    cudaError_t e =
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SmemLayout::kDynamic);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
   kern<<<grid, kThreads, SmemLayout::kDynamic, s>>>(p, a, b0, b1, bs0, bs1);
   return cudaGetLastError();
 }

@@ -74,7 +74,7 @@ def test_argument_errors_need_no_device(lib):
     # workspace too small / misaligned
     assert lib.moe_forward(ctypes.byref(cfg), 4, 1024, ctypes.byref(w), 2048, None, None, 4096, 16, None) == \
         m.MOE_ERR_WORKSPACE_TOO_SMALL
-    assert lib.moe_forward(ctypes.byref(cfg), 4, 1024, ctypes.byref(w), 2048, None, None, 4100, 1 << 30, None) == \
+    assert lib.moe_forward(ctypes.byref(cfg), 4, 1024, ctypes.byref(w), 2048, None, None, 4352 + 64, 1 << 30, None) == \
         m.MOE_ERR_MISALIGNED
     # only one of topk_idx / topk_w
     assert lib.moe_forward(ctypes.byref(cfg), 4, 1024, ctypes.byref(w), 2048, 4096, None, 8192, 1 << 30, None) == \

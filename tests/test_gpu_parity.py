@@ -109,8 +109,10 @@ def test_route_parity(m, shape):
     m.moe_route(cfg, T, m.to_device(x), m.to_device(wr), m.to_device(bias), idx, gate, logits, ws)
     assert m.moe_read_status(ws) == 0
     lg = logits.cpu().numpy().astype(np.float64)
+    # The routing comparison is sound while the fp32 logits stay within half the
+    # 1e-4 margin of the fp64 ones (fp32 accumulation over H = 4096 products).
     err = np.abs(lg - logits_r).max()
-    assert err < 2e-5, f"fp32 logits off by {err}"
+    assert err < 5e-5, f"fp32 logits off by {err}"
     n_u, n_a = check_routing(idx.cpu().numpy(), gate.cpu().numpy(), logits_r, idx_r, gate_r)
     assert n_u >= 0.99 * T
 
