@@ -8,7 +8,8 @@ returns an error; there is no fallback.
 The functions carry the names of the C entry points:
   moe_workspace_bytes, moe_forward, moe_forward_host, moe_route,
   moe_quantize_act, moe_permute, moe_experts, moe_combine, moe_read_status,
-  moe_status_string, moe_profile_enable, moe_profile_read, moe_device_sm_count.
+  moe_status_string, moe_profile_enable, moe_profile_read, moe_device_sm_count,
+  moe_set_gemm_variant.
 """
 from __future__ import annotations
 
@@ -28,6 +29,7 @@ MOE_ERR_CUDA = 4
 MOE_ERR_BAD_INDEX = 5
 MOE_ERR_DEVICE_TIMEOUT = 6
 MOE_ERR_MISALIGNED = 7
+MOE_GEMM_AUTO, MOE_GEMM_SINGLE, MOE_GEMM_PAIR = 0, 1, 2
 
 _lib = None
 
@@ -76,6 +78,7 @@ def load():
         "moe_profile_read": [ctypes.POINTER(ctypes.c_float), ctypes.c_int, ctypes.POINTER(ctypes.c_int)],
         "moe_profile_kernel_name": [ctypes.c_int],
         "moe_device_sm_count": [ctypes.POINTER(ctypes.c_int)],
+        "moe_set_gemm_variant": [ctypes.c_int],
     }
     for name, args in sig.items():
         f = getattr(lib, name)
@@ -185,6 +188,10 @@ def moe_profile_read() -> dict:
     _check(load().moe_profile_read(buf, 16, ctypes.byref(n)), "moe_profile_read")
     lib = load()
     return {lib.moe_profile_kernel_name(i).decode(): float(buf[i]) for i in range(n.value)}
+
+
+def moe_set_gemm_variant(variant: int):
+    _check(load().moe_set_gemm_variant(variant), "moe_set_gemm_variant")
 
 
 def moe_device_sm_count() -> int:

@@ -16,6 +16,11 @@ namespace {
 // CTAs the router aims for when it splits K for small token counts (B200: 148 SMs).
 constexpr int kRouterTargetCtas = 148;
 
+// The 2-SM (CTA pair) expert GEMMs pay off once expert groups average more
+// than this many rows (below it, the pair's second half is mostly padding).
+constexpr int64_t kPairMinRowsPerGroup = 100;
+int g_gemm_variant = MOE_GEMM_AUTO;
+
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 std::once_flag g_encode_once;
 
@@ -187,6 +192,7 @@ PermuteParams permute_params(const moe_config* c, const WsLayout& L, int64_t T, 
   pp.counts = reinterpret_cast<int32_t*>(ws + L.counts);
   pp.offsets = reinterpret_cast<int32_t*>(ws + L.offsets);
   pp.mt_prefix = reinterpret_cast<int32_t*>(ws + L.mt_prefix);
+  pp.mp_prefix = reinterpret_cast<int32_t*>(ws + L.mp_prefix);
   pp.perm = reinterpret_cast<int32_t*>(ws + L.perm);
   pp.pos = reinterpret_cast<int32_t*>(ws + L.pos);
   pp.row_gate = gate ? reinterpret_cast<float*>(ws + L.row_gate) : nullptr;
@@ -215,6 +221,8 @@ int run_experts(const moe_config* c, const WsLayout& L, int64_t T, const void* x
   const int64_t R = L.R;
   const int sms = sm_count();
   if (sms <= 0) return MOE_ERR_CUDA;
+  const bool pair = g_gemm_variant == MOE_GEMM_PAIR ||
+                    (g_gemm_variant == MOE_GEMM_AUTO && R >= kPairMinRowsPerGroup * (E + S));
 
   GatherParams gp{};
   gp.T = (int32_t)T;
@@ -246,7 +254,7 @@ int run_experts(const moe_config* c, const WsLayout& L, int64_t T, const void* x
   if (!ok) return MOE_ERR_CUDA;
 
   GemmParams g1{};
-  g1.mt_prefix = reinterpret_cast<const int32_t*>(ws + L.mt_prefix);
+  g1.mt_prefix = reinterpret_cast<const int32_t*>(ws + (pair ? L.mp_prefix : L.mt_prefix));
   g1.offsets = reinterpret_cast<const int32_t*>(ws + L.offsets);
   g1.G = E + S;
   g1.E = E;
@@ -264,7 +272,7 @@ int run_experts(const moe_config* c, const WsLayout& L, int64_t T, const void* x
   g1.out_scale = fp8 ? reinterpret_cast<float*>(ws + L.sh) : nullptr;
   g1.row_gate = nullptr;
   g1.status = reinterpret_cast<int*>(ws + L.status);
-  CUDA_TRY(launch_gemm1(g1, fp8, sms, m.xp, m.w1, m.w3, m.sw1, m.sw3, s));
+  CUDA_TRY(launch_gemm1(g1, fp8, pair, sms, m.xp, m.w1, m.w3, m.sw1, m.sw3, s));
   prof.mark();
 
   GemmParams g2 = g1;
@@ -279,7 +287,7 @@ int run_experts(const moe_config* c, const WsLayout& L, int64_t T, const void* x
   g2.out = y;
   g2.out_scale = nullptr;
   g2.row_gate = reinterpret_cast<const float*>(ws + L.row_gate);
-  CUDA_TRY(launch_gemm2(g2, fp8, sms, m.h, m.w2, m.sw2, s));
+  CUDA_TRY(launch_gemm2(g2, fp8, pair, sms, m.h, m.w2, m.sw2, s));
   prof.mark();
   return MOE_OK;
 }
@@ -315,7 +323,7 @@ WsLayout ws_layout(const moe_config& c, int64_t T, int target_ctas) {
   const int64_t es = fp8 ? 1 : 2;
   L.T = T;
   L.R = (int64_t)(k + S) * T;
-  L.rows_pad = round_up(L.R, kTileM) + kTileM;
+  L.rows_pad = round_up(L.R, kTileM) + 2 * kTileM;  // a 256-row pair tile may start at the last row
   L.chunks = ceil_div(T > 0 ? T : 1, kHistChunk);
   const int64_t m_tiles = ceil_div(T > 0 ? T : 1, kTileM);
   int64_t ks = target_ctas / m_tiles;
@@ -335,6 +343,7 @@ WsLayout ws_layout(const moe_config& c, int64_t T, int target_ctas) {
   L.counts = take((size_t)G * 4);
   L.offsets = take((size_t)(G + 1) * 4);
   L.mt_prefix = take((size_t)(G + 1) * 4);
+  L.mp_prefix = take((size_t)(G + 1) * 4);
   L.perm = take((size_t)L.R * 4);
   L.pos = take((size_t)T * (k + S) * 4);
   L.row_gate = take((size_t)L.R * 4);
@@ -545,6 +554,12 @@ int moe_profile_read(float* ms, int n, int* n_out) {
 }
 
 const char* moe_profile_kernel_name(int i) { return (i >= 0 && i < kProfKernels) ? kProfNames[i] : ""; }
+
+int moe_set_gemm_variant(int variant) {
+  if (variant != MOE_GEMM_AUTO && variant != MOE_GEMM_SINGLE && variant != MOE_GEMM_PAIR) return MOE_ERR_INVALID_ARG;
+  g_gemm_variant = variant;
+  return MOE_OK;
+}
 
 int moe_device_sm_count(int* sms) {
   if (!sms) return MOE_ERR_INVALID_ARG;

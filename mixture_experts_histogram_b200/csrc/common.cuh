@@ -24,7 +24,7 @@ __host__ __device__ inline int64_t round_up(int64_t a, int64_t b) { return ceil_
 // from its base; every buffer starts on a 1024-byte boundary).
 struct WsLayout {
   int64_t T, R, rows_pad, chunks, ksplit;
-  size_t status, idx, gate, logits_part, chunk_base, counts, offsets, mt_prefix;
+  size_t status, idx, gate, logits_part, chunk_base, counts, offsets, mt_prefix, mp_prefix;
   size_t perm, pos, row_gate, xp, sxp, h, sh, y, x_stage, out_stage, total;
 };
 
@@ -59,6 +59,7 @@ struct PermuteParams {
   int32_t* counts;          // [G]
   int32_t* offsets;         // [G + 1]
   int32_t* mt_prefix;       // [G + 1] M-tile prefix (tiles of kTileM rows)
+  int32_t* mp_prefix;       // [G + 1] pair-tile prefix (tiles of 2 kTileM rows, 2-SM GEMMs)
   int32_t* perm;            // [S T]
   int32_t* pos;             // [T, S]
   float* row_gate;          // [S T] or null
@@ -78,7 +79,7 @@ struct GatherParams {
 
 // ---- grouped expert GEMMs ----
 struct GemmParams {
-  const int32_t* mt_prefix;  // [G + 1]
+  const int32_t* mt_prefix;  // [G + 1] tile prefix (128-row tiles, or 256-row pair tiles)
   const int32_t* offsets;    // [G + 1]
   int32_t G, E;              // groups, routed experts (group E is the shared expert)
   int32_t K, N;              // reduction length; output width (I for GEMM1, H for GEMM2)
@@ -111,10 +112,12 @@ cudaError_t launch_histogram(const PermuteParams& p, cudaStream_t s);
 cudaError_t launch_scan(const PermuteParams& p, cudaStream_t s);
 cudaError_t launch_scatter(const PermuteParams& p, cudaStream_t s);
 cudaError_t launch_gather(const GatherParams& p, bool fp8, cudaStream_t s);
-cudaError_t launch_gemm1(const GemmParams& p, bool fp8, int grid, const CUtensorMap& tm_a,
+// pair: run the 2-SM (CTA pair, M = 256) variant; p.mt_prefix must then be the
+// pair-tile prefix and `grid` even.
+cudaError_t launch_gemm1(const GemmParams& p, bool fp8, bool pair, int grid, const CUtensorMap& tm_a,
                          const CUtensorMap& tm_w1, const CUtensorMap& tm_w3, const CUtensorMap& tm_sw1,
                          const CUtensorMap& tm_sw3, cudaStream_t s);
-cudaError_t launch_gemm2(const GemmParams& p, bool fp8, int grid, const CUtensorMap& tm_a,
+cudaError_t launch_gemm2(const GemmParams& p, bool fp8, bool pair, int grid, const CUtensorMap& tm_a,
                          const CUtensorMap& tm_w2, const CUtensorMap& tm_sw2, cudaStream_t s);
 cudaError_t launch_combine(const CombineParams& p, cudaStream_t s);
 

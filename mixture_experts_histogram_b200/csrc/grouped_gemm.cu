@@ -12,20 +12,31 @@
 //     codes E4M3, scales stored transposed [I/128, rows].
 //   GEMM2 (down):  y[r, c] = gate[r] * (h[r] . W2_g[c]), stored bf16.
 //
-// Tiles: 128 rows x 256 accumulator columns. GEMM1 puts 128 gate columns (W1
-// rows n0..n0+127) and the matching 128 up columns (W3 rows n0..n0+127) side by
-// side in one N = 256 MMA, so SwiGLU pairs sit in one thread's registers. GEMM2
-// covers 256 output columns.
+// Accumulator tile per CTA: 128 rows x 256 columns. GEMM1's 256 columns are
+// 128 gate columns (W1 rows n0..n0+127) and the matching 128 up columns (W3
+// rows n0..n0+127) side by side in one N = 256 MMA, so SwiGLU pairs sit in one
+// thread's registers. GEMM2 covers 256 output columns.
 //
-// Persistent CTAs (one per SM) walk a static list of work items; an item is
+// Two variants:
+//   single (kPair = false): one CTA per tile; each stage holds A (128 rows) and
+//     the whole 256-row B tile (48 KB); 4 stages.
+//   pair (kPair = true): a cluster of two CTAs on one TPC computes a 256-row
+//     tile with 2-SM MMAs (M = 256). Each CTA loads its own 128 A rows and one
+//     128-row half of the B tile (32 KB a stage, 6 stages), so every weight
+//     tile crosses L2 -> SM once per pair instead of once per 128 rows: a third
+//     less L2 traffic per FLOP, for groups with more than ~100 rows.
+//
+// Persistent CTAs (pairs) walk a static list of work items; an item is
 // (group, N tile, M tile) with the M tiles of one (group, N tile) adjacent, so
 // CTAs that share a weight tile run together and the second read hits L2.
 // Warp roles:
-//   warp 0      TMA producer: A tile (128 rows x 128 B) + B tile (256 rows x 128 B)
-//               per stage into a 4-deep ring (128B swizzle).
-//   warp 1      allocates 512 TMEM columns; one thread issues the MMAs.
-//   warps 2-9   epilogue: each thread owns one row (TMEM lane) and one half of
-//               the tile's columns.
+//   warp 0      producer. Lane 0 issues the TMA loads. In FP8 mode all 32 lanes
+//               also cp.async each K block's 128 row scales and two
+//               weight-block scales into an 8-slot ring in shared memory.
+//   warp 1      allocates 512 TMEM columns; one thread issues the MMAs (in the
+//               pair variant only the even CTA of the pair issues them).
+//   warps 2-9   epilogue: 2 column halves x 4 TMEM lane quarters; each thread
+//               owns one row (TMEM lane) and one half of the tile's columns.
 // BF16: the accumulator lives in TMEM for the whole K loop; two 256-column
 // buffers let the epilogue of one tile overlap the MMAs of the next.
 // FP8: the fp32 block scales are not powers of two, so each 128-deep K block is
@@ -41,29 +52,42 @@ namespace moe {
 
 namespace {
 
-constexpr int kThreads = 320;
-constexpr int kStages = 4;
-constexpr int kABytes = kTileM * kStageBytesK;  // 16 KB
-constexpr int kBBytes = 256 * kStageBytesK;     // 32 KB
-constexpr int kStageBytes = kABytes + kBBytes;
+constexpr int kEpiWarps = 8;
+constexpr int kEpiThreads = kEpiWarps * 32;
+constexpr int kThreads = 64 + kEpiThreads;
+constexpr int kABytes = kTileM * kStageBytesK;  // 16 KB: 128 rows of A
+constexpr int kMaxStages = 6;
 constexpr int kMaxGroups = kMaxExperts + 1;
+constexpr int kScRing = 8;                      // K blocks of staged FP8 scales
+constexpr int kScSlot = 132;                    // floats: 128 row scales + 2 block scales (+ pad)
+#ifndef MOE_FP8_CHUNK
+#define MOE_FP8_CHUNK 16
+#endif
+constexpr int kFp8Chunk = MOE_FP8_CHUNK;        // TMEM columns per load when promoting FP8 partials
 
-struct SmemLayout {
+template <bool kPair>
+struct Cfg {
+  static constexpr int kStages = kPair ? 6 : 4;
+  static constexpr int kBBytes = (kPair ? 128 : 256) * kStageBytesK;  // this CTA's share of the B tile
+  static constexpr int kStageBytes = kABytes + kBBytes;
+  static constexpr int kTileRows = kPair ? 2 * kTileM : kTileM;      // rows of one work item
   static constexpr size_t kTiles = (size_t)kStages * kStageBytes;
-  static constexpr size_t kBars = kTiles;                              // full[4], empty[4], tfull[2], tempty[2], drain
-  static constexpr size_t kMisc = kBars + 16 * 8;                      // tmem slot, abort flag
-  static constexpr size_t kAmax = kMisc + 64;                          // float [2][2][128]
-  static constexpr size_t kMt = kAmax + 2 * 2 * 128 * 4;               // int [kMaxGroups + 1]
-  static constexpr size_t kOff = kMt + (kMaxGroups + 1) * 4;           // int [kMaxGroups + 1]
+  static constexpr size_t kScales = kTiles;                           // float [kScRing][kScSlot]
+  static constexpr size_t kBars = kScales + kScRing * kScSlot * 4;    // 2 kMaxStages + 5 + 2 kScRing barriers
+  static constexpr size_t kMisc = kBars + 256;                        // tmem slot, abort flag
+  static constexpr size_t kAmax = kMisc + 64;                         // float [2][2][128]
+  static constexpr size_t kMt = kAmax + 2 * 2 * 128 * 4;              // int [kMaxGroups + 1]
+  static constexpr size_t kOff = kMt + (kMaxGroups + 1) * 4;          // int [kMaxGroups + 1]
   static constexpr size_t kEnd = kOff + (kMaxGroups + 1) * 4;
-  static constexpr size_t kDynamic = kEnd + 1024;                      // + alignment slack
+  static constexpr size_t kDynamic = kEnd + 1024;                     // + alignment slack
 };
 
 struct Item {
-  int g, n, row0, valid;
+  int g, n, row0, end;  // group, N tile, first row of the tile, end of the group's rows
 };
 
-__device__ __forceinline__ Item decode_item(int item, int n_tiles, int G, const int* s_mt, const int* s_off) {
+__device__ __forceinline__ Item decode_item(int item, int n_tiles, int G, int tile_rows, const int* s_mt,
+                                            const int* s_off) {
   const int q = item / n_tiles;
   int lo = 0, hi = G;  // s_mt[lo] <= q < s_mt[hi]
   while (hi - lo > 1) {
@@ -76,11 +100,26 @@ __device__ __forceinline__ Item decode_item(int item, int n_tiles, int G, const 
   const int mtiles = s_mt[lo + 1] - s_mt[lo];
   const int local = item - n_tiles * s_mt[lo];
   it.n = local / mtiles;
-  const int m = local % mtiles;
-  it.row0 = s_off[lo] + m * kTileM;
-  it.valid = min(kTileM, s_off[lo + 1] - it.row0);
+  it.row0 = s_off[lo] + (local % mtiles) * tile_rows;
+  it.end = s_off[lo + 1];
   return it;
 }
+
+// Weight-tile rows of a work item: box 0 starts at row `yb` of `*m0`, box 1 at
+// row `yb2` of `*m1` (GEMM1: W1 and W3 rows n0..; GEMM2: W2 rows n0.. and n0+128..).
+template <bool kGemm1>
+struct BRows {
+  const CUtensorMap *m0, *m1;
+  int yb, yb2;
+  __device__ __forceinline__ BRows(const Item& it, const GemmParams& p, const CUtensorMap* b0, const CUtensorMap* b1,
+                                   const CUtensorMap* bs0, const CUtensorMap* bs1) {
+    const bool shared = (it.g == p.E);
+    yb = (shared ? 0 : it.g * p.N) + it.n * (kGemm1 ? 128 : 256);
+    m0 = shared ? bs0 : b0;
+    m1 = kGemm1 ? (shared ? bs1 : b1) : m0;
+    yb2 = kGemm1 ? yb : yb + 128;
+  }
+};
 
 __device__ __forceinline__ float silu_mul(float g, float u) { return g / (1.0f + __expf(-g)) * u; }
 
@@ -91,48 +130,61 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
 
 // Bounded wait by every lane, with a warp-uniform verdict (keeps the warp
 // converged for the .sync.aligned TMEM loads that follow).
+template <bool kCluster>
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, int* status, volatile int* abort_flag) {
-  const bool ok = mbar_wait(bar, parity, status, abort_flag);
+  const bool ok = kCluster ? mbar_wait_cluster(bar, parity, status, abort_flag)
+                           : mbar_wait(bar, parity, status, abort_flag);
   return __all_sync(0xffffffffu, ok);
 }
 
-template <bool kFP8, bool kGemm1>
+template <bool kFP8, bool kGemm1, bool kPair>
 __global__ void __launch_bounds__(kThreads, 1)
     grouped_gemm_kernel(const GemmParams p, const __grid_constant__ CUtensorMap tm_a,
                         const __grid_constant__ CUtensorMap tm_b0, const __grid_constant__ CUtensorMap tm_b1,
                         const __grid_constant__ CUtensorMap tm_bs0, const __grid_constant__ CUtensorMap tm_bs1) {
+  using C = Cfg<kPair>;
   constexpr int kElemsPerStage = kFP8 ? 128 : 64;  // 128 bytes of K per stage
-  constexpr uint32_t kIdesc = idesc_mma(kFP8 ? 0u : 1u, kTileM, 256);
+  constexpr uint32_t kIdesc = idesc_mma(kFP8 ? 0u : 1u, kPair ? 2 * kTileM : kTileM, 256);
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
-  uint8_t* sB = smem + kStages * kABytes;
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + SmemLayout::kBars);
-  uint64_t* empty = full + kStages;
-  uint64_t* tfull = empty + kStages;
+  uint8_t* sB = smem + C::kStages * kABytes;
+  float* sc = reinterpret_cast<float*>(smem + C::kScales);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kBars);
+  uint64_t* empty = full + kMaxStages;
+  uint64_t* tfull = empty + kMaxStages;
   uint64_t* tempty = tfull + 2;
   uint64_t* drain = tempty + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + SmemLayout::kMisc);
+  uint64_t* scfull = drain + 1;
+  uint64_t* scempty = scfull + kScRing;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  float* amax_x = reinterpret_cast<float*>(smem + SmemLayout::kAmax);
-  int* s_mt = reinterpret_cast<int*>(smem + SmemLayout::kMt);
-  int* s_off = reinterpret_cast<int*>(smem + SmemLayout::kOff);
+  float* amax_x = reinterpret_cast<float*>(smem + C::kAmax);
+  int* s_mt = reinterpret_cast<int*>(smem + C::kMt);
+  int* s_off = reinterpret_cast<int*>(smem + C::kOff);
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const uint32_t rank = kPair ? cluster_cta_rank() : 0u;  // 0 = the pair's MMA issuer
+  const int unit = kPair ? (int)(blockIdx.x / 2) : (int)blockIdx.x;
+  const int n_units = kPair ? (int)(gridDim.x / 2) : (int)gridDim.x;
 
   for (int i = threadIdx.x; i <= p.G; i += kThreads) {
     s_mt[i] = p.mt_prefix[i];
     s_off[i] = p.offsets[i];
   }
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kStages; ++s) {
+    for (int s = 0; s < C::kStages; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&tfull[b], 1);
-      mbar_init(&tempty[b], 256);
+      mbar_init(&tempty[b], kPair ? 2 * kEpiThreads : kEpiThreads);
+    }
+    for (int j = 0; j < kScRing; ++j) {
+      mbar_init(&scfull[j], 32);
+      mbar_init(&scempty[j], kEpiThreads);
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -148,98 +200,162 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, 512);
-    tmem_relinquish();
+    if (kPair) {
+      tmem_alloc_pair(tmem_slot, 512);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(tmem_slot, 512);
+      tmem_relinquish();
+    }
   }
   __syncthreads();
+  if (kPair) cluster_sync();  // the peer's barriers are initialised before any remote arrive
   tc_fence_after_sync();
   const uint32_t tmem = *tmem_slot;
   const int total = s_mt[p.G] * p.n_tiles;
   const int kstages = p.K / kElemsPerStage;
+  const int nkb = p.K / 128;
+  const int my_off = kPair ? kTileM * (int)rank : 0;  // this CTA's rows inside a work item
 
   if (warp == 0) {
-    if (lane == 0) {
-      // ---------------------------------------------------- TMA producer --
-      int stage = 0;
-      uint32_t phase = 0;
-      uint32_t issued = 0;  // bit s: stage s has a load in flight at phase bit (issued_phase >> s) & 1
-      uint32_t issued_phase = 0;
-      bool ok = true;
-      for (int item = blockIdx.x; item < total && ok; item += gridDim.x) {
-        const Item it = decode_item(item, p.n_tiles, p.G, s_mt, s_off);
-        const bool shared = (it.g == p.E);
-        int yb;
-        if (kGemm1) yb = (shared ? 0 : it.g * p.N) + it.n * 128;
-        else yb = (shared ? 0 : it.g * p.N) + it.n * 256;
-        const CUtensorMap* mb0 = shared ? &tm_bs0 : &tm_b0;
-        const CUtensorMap* mb1 = kGemm1 ? (shared ? &tm_bs1 : &tm_b1) : mb0;
-        for (int ks = 0; ks < kstages; ++ks) {
-          if (!mbar_wait(&empty[stage], phase ^ 1, p.status, abort_flag)) { ok = false; break; }
-          mbar_arrive_expect_tx(&full[stage], kStageBytes);
-          const int kx = ks * kElemsPerStage;
-          tma_load_2d(sA + stage * kABytes, &tm_a, &full[stage], kx, it.row0);
-          tma_load_2d(sB + stage * kBBytes, mb0, &full[stage], kx, yb);
-          tma_load_2d(sB + stage * kBBytes + kBBytes / 2, mb1, &full[stage], kx, kGemm1 ? yb : yb + 128);
-          issued |= 1u << stage;
-          issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
-          if (++stage == kStages) { stage = 0; phase ^= 1; }
+    // ------------------------------------------------------------ producer --
+    int stage = 0;
+    uint32_t phase = 0, sc_iter = 0;
+    uint32_t issued = 0;        // bit s: stage s has had a load issued
+    uint32_t issued_phase = 0;  // bit s: the phase of that last issue
+    bool ok = true;
+    for (int item = unit; item < total && ok; item += n_units) {
+      const Item it = decode_item(item, p.n_tiles, p.G, C::kTileRows, s_mt, s_off);
+      const bool shared = (it.g == p.E);
+      const int my_row0 = it.row0 + my_off;
+      const BRows<kGemm1> rows(it, p, &tm_b0, &tm_b1, &tm_bs0, &tm_bs1);
+      // FP8: where this tile's weight-block scales start (one fp32 per K block).
+      const float *sb0 = nullptr, *sb1 = nullptr;
+      if (kFP8) {
+        const int nblk = p.N / 128;
+        if (kGemm1) {
+          const int64_t blk = shared ? (int64_t)it.n : (int64_t)it.g * nblk + it.n;
+          sb0 = (shared ? p.bs_scale0 : p.b_scale0) + blk * nkb;
+          sb1 = (shared ? p.bs_scale1 : p.b_scale1) + blk * nkb;
+        } else {
+          const int nb0 = 2 * it.n, nb1 = (2 * it.n + 1 < nblk) ? 2 * it.n + 1 : 2 * it.n;
+          const float* base = shared ? p.bs_scale0 : p.b_scale0;
+          const int64_t g0 = shared ? 0 : (int64_t)it.g * nblk;
+          sb0 = base + (g0 + nb0) * nkb;
+          sb1 = base + (g0 + nb1) * nkb;
         }
       }
-      if (!ok) {
-        // Let the copies already in flight land before the CTA leaves.
-        for (int s = 0; s < kStages; ++s) {
-          if (!(issued & (1u << s))) continue;
-          const uint64_t t0 = global_timer_ns();
-          while (!mbar_try_wait(&full[s], (issued_phase >> s) & 1u) && global_timer_ns() - t0 < 200000000ull) {}
+      for (int ks = 0; ks < kstages; ++ks) {
+        bool w = true;
+        if (lane == 0) w = mbar_wait(&empty[stage], phase ^ 1, p.status, abort_flag);
+        if (!__shfl_sync(0xffffffffu, w ? 1 : 0, 0)) { ok = false; break; }
+        if (lane == 0) {
+          const int kx = ks * kElemsPerStage;
+          if (kPair) {
+            // Both CTAs' tiles complete on the even CTA's barrier, which expects them all.
+            const uint32_t bar0 = map_to_cta(&full[stage], 0);
+            if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2 * C::kStageBytes);
+            tma_load_2d_pair(sA + stage * kABytes, &tm_a, bar0, kx, my_row0);
+            tma_load_2d_pair(sB + stage * C::kBBytes, rank ? rows.m1 : rows.m0, bar0, kx, rank ? rows.yb2 : rows.yb);
+          } else {
+            mbar_arrive_expect_tx(&full[stage], C::kStageBytes);
+            tma_load_2d(sA + stage * kABytes, &tm_a, &full[stage], kx, my_row0);
+            tma_load_2d(sB + stage * C::kBBytes, rows.m0, &full[stage], kx, rows.yb);
+            tma_load_2d(sB + stage * C::kBBytes + C::kBBytes / 2, rows.m1, &full[stage], kx, rows.yb2);
+          }
+          issued |= 1u << stage;
+          issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
         }
+        if (kFP8) {
+          const uint32_t j = sc_iter % kScRing, sph = (sc_iter / kScRing) & 1u;
+          if (!warp_wait<false>(&scempty[j], sph ^ 1u, p.status, abort_flag)) { ok = false; break; }
+          float* slot = sc + j * kScSlot;
+          const float* src = p.a_scale + (int64_t)ks * p.rows_pad + my_row0 + lane * 4;
+#pragma unroll
+          for (int i = 0; i < 4; ++i) cp_async_4(slot + lane * 4 + i, src + i);
+          if (lane == 0) {
+            cp_async_4(slot + 128, sb0 + ks);
+            cp_async_4(slot + 129, sb1 + ks);
+          }
+          cp_async_arrive(&scfull[j]);
+          ++sc_iter;
+        }
+        if (++stage == C::kStages) { stage = 0; phase ^= 1; }
+      }
+    }
+    if (kFP8) asm volatile("cp.async.wait_all;" ::: "memory");
+    if (!ok && lane == 0 && rank == 0) {
+      // Let the tensor copies already in flight land before the CTA leaves.
+      for (int s = 0; s < C::kStages; ++s) {
+        if (!(issued & (1u << s))) continue;
+        const uint64_t t0 = global_timer_ns();
+        while (!mbar_try_wait(&full[s], (issued_phase >> s) & 1u) && global_timer_ns() - t0 < 200000000ull) {}
       }
     }
   } else if (warp == 1) {
-    if (lane == 0) {
+    if (lane == 0 && rank == 0) {
       // ------------------------------------------------------ MMA issuer --
+      auto mma = [&](uint32_t d, uint64_t ad, uint64_t bd, uint32_t acc) {
+        if (kPair) {
+          if (kFP8) mma_e4m3_pair(d, ad, bd, kIdesc, acc);
+          else mma_bf16_pair(d, ad, bd, kIdesc, acc);
+        } else {
+          if (kFP8) mma_e4m3(d, ad, bd, kIdesc, acc);
+          else mma_bf16(d, ad, bd, kIdesc, acc);
+        }
+      };
+      auto commit = [&](uint64_t* bar) {
+        if (kPair) mma_commit_pair(bar, 0x3);
+        else mma_commit(bar);
+      };
+      auto wait_tempty = [&](uint32_t b, uint32_t par) {
+        return kPair ? mbar_wait_cluster(&tempty[b], par, p.status, abort_flag)
+                     : mbar_wait(&tempty[b], par, p.status, abort_flag);
+      };
       int stage = 0;
       uint32_t phase = 0;
       uint32_t acc_iter = 0;
       bool ok = true;
-      for (int item = blockIdx.x; item < total && ok; item += gridDim.x) {
+      for (int item = unit; item < total && ok; item += n_units) {
         if (!kFP8) {
           const uint32_t b = acc_iter & 1u, tph = (acc_iter >> 1) & 1u;
-          if (!mbar_wait(&tempty[b], tph ^ 1u, p.status, abort_flag)) { ok = false; break; }
+          if (!wait_tempty(b, tph ^ 1u)) { ok = false; break; }
           tc_fence_after_sync();
           const uint32_t d = tmem + b * 256;
           for (int ks = 0; ks < kstages; ++ks) {
             if (!mbar_wait(&full[stage], phase, p.status, abort_flag)) { ok = false; break; }
             tc_fence_after_sync();
             const uint64_t ad = sdesc_k_sw128(sA + stage * kABytes);
-            const uint64_t bd = sdesc_k_sw128(sB + stage * kBBytes);
+            const uint64_t bd = sdesc_k_sw128(sB + stage * C::kBBytes);
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk) mma_bf16(d, ad + 2 * kk, bd + 2 * kk, kIdesc, (ks | kk) ? 1u : 0u);
-            mma_commit(&empty[stage]);
-            if (++stage == kStages) { stage = 0; phase ^= 1; }
+            for (int kk = 0; kk < 4; ++kk) mma(d, ad + 2 * kk, bd + 2 * kk, (ks | kk) ? 1u : 0u);
+            commit(&empty[stage]);
+            if (++stage == C::kStages) { stage = 0; phase ^= 1; }
           }
           if (!ok) break;
-          mma_commit(&tfull[b]);
+          commit(&tfull[b]);
           ++acc_iter;
         } else {
           for (int ks = 0; ks < kstages; ++ks) {
             const uint32_t b = acc_iter & 1u, tph = (acc_iter >> 1) & 1u;
-            if (!mbar_wait(&tempty[b], tph ^ 1u, p.status, abort_flag)) { ok = false; break; }
+            if (!wait_tempty(b, tph ^ 1u)) { ok = false; break; }
             if (!mbar_wait(&full[stage], phase, p.status, abort_flag)) { ok = false; break; }
             tc_fence_after_sync();
             const uint32_t d = tmem + b * 256;
             const uint64_t ad = sdesc_k_sw128(sA + stage * kABytes);
-            const uint64_t bd = sdesc_k_sw128(sB + stage * kBBytes);
+            const uint64_t bd = sdesc_k_sw128(sB + stage * C::kBBytes);
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk) mma_e4m3(d, ad + 2 * kk, bd + 2 * kk, kIdesc, kk ? 1u : 0u);
-            mma_commit(&empty[stage]);
-            mma_commit(&tfull[b]);
+            for (int kk = 0; kk < 4; ++kk) mma(d, ad + 2 * kk, bd + 2 * kk, kk ? 1u : 0u);
+            commit(&empty[stage]);
+            commit(&tfull[b]);
             ++acc_iter;
-            if (++stage == kStages) { stage = 0; phase ^= 1; }
+            if (++stage == C::kStages) { stage = 0; phase ^= 1; }
           }
         }
       }
       // Drain: every MMA issued so far has completed once this arrives.
-      mma_commit(drain);
+      if (kPair) mma_commit_pair(drain, 0x1);
+      else mma_commit(drain);
       const uint64_t t0 = global_timer_ns();
       while (!mbar_try_wait(drain, 0) && global_timer_ns() - t0 < 200000000ull) {}
     }
@@ -247,145 +363,144 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ---------------------------------------------------------- epilogue --
     const int q = warp % 4;            // TMEM lane quarter this warp may read
     const int hf = (warp - 2) / 4;     // which half of the tile's columns
-    const int rl = q * 32 + lane;      // row inside the tile
+    const int rl = q * 32 + lane;      // row inside this CTA's 128 rows
     const uint32_t lane_base = (uint32_t)(q * 32) << 16;
-    uint32_t acc_iter = 0, tile_iter = 0;
+    // The accumulator is released on the pair's even CTA (or locally).
+    auto release_acc = [&](uint32_t b) {
+      tc_fence_before_sync();
+      if (kPair) mbar_arrive_cluster(map_to_cta(&tempty[b], 0));
+      else mbar_arrive(&tempty[b]);
+    };
+    uint32_t acc_iter = 0, tile_iter = 0, sc_iter = 0;
     bool ok = true;
-    const int nkb = p.K / 128;
-    for (int item = blockIdx.x; item < total; item += gridDim.x) {
-      const Item it = decode_item(item, p.n_tiles, p.G, s_mt, s_off);
-      const bool shared = (it.g == p.E);
-      const int64_t row = (int64_t)it.row0 + rl;
-      const bool row_ok = rl < it.valid;
+    for (int item = unit; item < total; item += n_units) {
+      const Item it = decode_item(item, p.n_tiles, p.G, C::kTileRows, s_mt, s_off);
+      const int64_t row = (int64_t)it.row0 + my_off + rl;
+      const bool row_ok = row < it.end;
+      // Output columns of this thread: GEMM1 h columns n*128 + 64 hf (+64);
+      // GEMM2 y columns n*256 + 128 hf (+128).
+      const int col0 = kGemm1 ? it.n * 128 + 64 * hf : it.n * 256 + 128 * hf;
+      const bool col_ok = col0 < p.N;
       if (!kFP8) {
         const uint32_t b = acc_iter & 1u, tph = (acc_iter >> 1) & 1u;
-        if (ok) ok = warp_wait(&tfull[b], tph, p.status, abort_flag);
+        if (ok) ok = warp_wait<kPair>(&tfull[b], tph, p.status, abort_flag);
         tc_fence_after_sync();
         const uint32_t base = tmem + lane_base + b * 256;
         if (kGemm1) {
-          uint16_t* hout = static_cast<uint16_t*>(p.out);
 #pragma unroll
           for (int ch = 0; ch < 2; ++ch) {
             uint32_t g[32], u[32];
-            tmem_ld32(base + hf * 64 + ch * 32, g);
-            tmem_ld32(base + 128 + hf * 64 + ch * 32, u);
+            tmem_ld32(base + 64 * hf + 32 * ch, g);
+            tmem_ld32(base + 128 + 64 * hf + 32 * ch, u);
             tmem_ld_wait();
+            if (ch == 1) release_acc(b);
             uint32_t pk[16];
 #pragma unroll
             for (int i = 0; i < 16; ++i)
               pk[i] = pack_bf16x2(silu_mul(__uint_as_float(g[2 * i]), __uint_as_float(u[2 * i])),
                                   silu_mul(__uint_as_float(g[2 * i + 1]), __uint_as_float(u[2 * i + 1])));
             if (ok && row_ok) {
-              uint4* dst = reinterpret_cast<uint4*>(hout + row * p.N + it.n * 128 + hf * 64 + ch * 32);
+              uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.out) + row * p.N + col0 + 32 * ch);
 #pragma unroll
               for (int v = 0; v < 4; ++v) dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
             }
           }
         } else {
-          uint16_t* yout = static_cast<uint16_t*>(p.out);
           const float gw = row_ok ? p.row_gate[row] : 0.0f;
-          const int col0 = it.n * 256 + hf * 128;
 #pragma unroll
           for (int ch = 0; ch < 4; ++ch) {
             uint32_t v[32];
-            tmem_ld32(base + hf * 128 + ch * 32, v);
+            tmem_ld32(base + 128 * hf + 32 * ch, v);
             tmem_ld_wait();
+            if (ch == 3) release_acc(b);
             uint32_t pk[16];
 #pragma unroll
             for (int i = 0; i < 16; ++i)
               pk[i] = pack_bf16x2(__uint_as_float(v[2 * i]) * gw, __uint_as_float(v[2 * i + 1]) * gw);
-            if (ok && row_ok && col0 < p.N) {
-              uint4* dst = reinterpret_cast<uint4*>(yout + row * p.N + col0 + ch * 32);
+            if (ok && row_ok && col_ok) {
+              uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.out) + row * p.N + col0 + 32 * ch);
 #pragma unroll
               for (int w = 0; w < 4; ++w) dst[w] = make_uint4(pk[4 * w], pk[4 * w + 1], pk[4 * w + 2], pk[4 * w + 3]);
             }
           }
         }
-        tc_fence_before_sync();
-        mbar_arrive(&tempty[b]);
         ++acc_iter;
       } else {
         // FP8: promote each K block's partial with its two block scales.
         float2 acc[64];
 #pragma unroll
         for (int i = 0; i < 64; ++i) acc[i] = make_float2(0.0f, 0.0f);
-        const float* sa = p.a_scale + row;
-        const float *sb0, *sb1;
-        if (kGemm1) {
-          const int64_t blk = shared ? (int64_t)it.n : ((int64_t)it.g * (p.N / 128) + it.n);
-          sb0 = (shared ? p.bs_scale0 : p.b_scale0) + blk * nkb;
-          sb1 = (shared ? p.bs_scale1 : p.b_scale1) + blk * nkb;
-        } else {
-          const int nb = it.n * 2 + hf;
-          const int64_t blk = shared ? (int64_t)nb : ((int64_t)it.g * (p.N / 128) + nb);
-          sb0 = (shared ? p.bs_scale0 : p.b_scale0) + blk * nkb;
-          sb1 = sb0;
-        }
-        const bool col_ok = kGemm1 || (it.n * 256 + hf * 128 < p.N);
         for (int kb = 0; kb < nkb; ++kb) {
+          const uint32_t j = sc_iter % kScRing, sph = (sc_iter / kScRing) & 1u;
+          if (ok) ok = warp_wait<false>(&scfull[j], sph, p.status, abort_flag);
+          const float* slot = sc + j * kScSlot;
+          const float a_s = slot[rl];
+          const float s0 = slot[128], s1 = slot[129];
+          mbar_arrive(&scempty[j]);
+          ++sc_iter;
+          // GEMM1: the first 64 columns are gate columns (s0), the next 64 up columns (s1).
+          // GEMM2: the half's 128 columns sit in n-block 2n (hf 0, s0) or 2n+1 (s1).
+          const float f0 = a_s * ((kGemm1 || hf == 0) ? s0 : s1);
+          const float f1 = kGemm1 ? a_s * s1 : f0;
           const uint32_t b = acc_iter & 1u, tph = (acc_iter >> 1) & 1u;
-          const float a_s = sa[(int64_t)kb * p.rows_pad];
-          const float f0 = a_s * (col_ok ? sb0[kb] : 0.0f);
-          const float f1 = kGemm1 ? a_s * sb1[kb] : f0;
-          if (ok) ok = warp_wait(&tfull[b], tph, p.status, abort_flag);
+          if (ok) ok = warp_wait<kPair>(&tfull[b], tph, p.status, abort_flag);
           tc_fence_after_sync();
           const uint32_t base = tmem + lane_base + b * 256;
+          constexpr int kNch = 128 / kFp8Chunk;  // chunks per thread per K block
 #pragma unroll
-          for (int ch = 0; ch < 4; ++ch) {
-            uint32_t v[32];
-            // GEMM1: chunks 0,1 = gate columns, 2,3 = up columns of this half.
-            const uint32_t col = kGemm1 ? ((ch < 2 ? 0u : 128u) + hf * 64 + (ch & 1) * 32) : (hf * 128 + ch * 32);
-            tmem_ld32(base + col, v);
+          for (int ch = 0; ch < kNch; ++ch) {
+            uint32_t v[kFp8Chunk];
+            const int c = ch * kFp8Chunk;  // 0..127 within this thread's 128 columns
+            const uint32_t col = kGemm1 ? (c < 64 ? 0u : 128u) + 64 * hf + (c & 63) : 128 * hf + c;
+            if constexpr (kFp8Chunk == 32) tmem_ld32(base + col, v);
+            else tmem_ld16(base + col, v);
             tmem_ld_wait();
-            const float f = (kGemm1 && ch >= 2) ? f1 : f0;
+            if (ch == kNch - 1) release_acc(b);
+            const float f = (kGemm1 && c >= 64) ? f1 : f0;
             const float2 ff = make_float2(f, f);
 #pragma unroll
-            for (int i = 0; i < 16; ++i)
-              acc[ch * 16 + i] = fma2(make_float2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1])), ff,
-                                      acc[ch * 16 + i]);
+            for (int i = 0; i < kFp8Chunk / 2; ++i)
+              acc[c / 2 + i] = fma2(make_float2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1])), ff,
+                                    acc[c / 2 + i]);
           }
-          tc_fence_before_sync();
-          mbar_arrive(&tempty[b]);
           ++acc_iter;
         }
         if (kGemm1) {
-          // SwiGLU, then the 1x128 block quantisation of h (the block spans both halves).
-          float hv[64];
+          // SwiGLU in place (acc[0..31] gate, acc[32..63] up), then the 1x128 block
+          // quantisation of h; the block spans both column halves.
           float amax = 0.0f;
 #pragma unroll
           for (int i = 0; i < 32; ++i) {
-            hv[2 * i] = silu_mul(acc[i].x, acc[32 + i].x);
-            hv[2 * i + 1] = silu_mul(acc[i].y, acc[32 + i].y);
-            amax = fmaxf(amax, fmaxf(fabsf(hv[2 * i]), fabsf(hv[2 * i + 1])));
+            acc[i].x = silu_mul(acc[i].x, acc[32 + i].x);
+            acc[i].y = silu_mul(acc[i].y, acc[32 + i].y);
+            amax = fmaxf(amax, fmaxf(fabsf(acc[i].x), fabsf(acc[i].y)));
           }
           float* ax = amax_x + (tile_iter & 1u) * 256;
           ax[hf * 128 + rl] = amax;
-          named_bar_sync(1, 256);
+          named_bar_sync(1, kEpiThreads);
           amax = fmaxf(amax, ax[(1 - hf) * 128 + rl]);
           const float s = amax > 0.0f ? __fdiv_rn(amax, 448.0f) : 1.0f;
           const float inv = amax > 0.0f ? __frcp_rn(s) : 0.0f;
           uint32_t pk[16];
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
-            const uint32_t lo = __nv_cvt_float2_to_fp8x2(make_float2(hv[4 * i] * inv, hv[4 * i + 1] * inv),
+            const uint32_t lo = __nv_cvt_float2_to_fp8x2(make_float2(acc[2 * i].x * inv, acc[2 * i].y * inv),
                                                          __NV_SATFINITE, __NV_E4M3);
-            const uint32_t hi = __nv_cvt_float2_to_fp8x2(make_float2(hv[4 * i + 2] * inv, hv[4 * i + 3] * inv),
-                                                         __NV_SATFINITE, __NV_E4M3);
+            const uint32_t hi = __nv_cvt_float2_to_fp8x2(
+                make_float2(acc[2 * i + 1].x * inv, acc[2 * i + 1].y * inv), __NV_SATFINITE, __NV_E4M3);
             pk[i] = lo | (hi << 16);
           }
           if (ok && row_ok) {
-            uint8_t* hout = static_cast<uint8_t*>(p.out);
-            uint4* dst = reinterpret_cast<uint4*>(hout + row * p.N + it.n * 128 + hf * 64);
+            uint4* dst = reinterpret_cast<uint4*>(static_cast<uint8_t*>(p.out) + row * p.N + col0);
 #pragma unroll
             for (int v = 0; v < 4; ++v) dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
             if (hf == 0) p.out_scale[(int64_t)it.n * p.rows_pad + row] = s;
           }
           ++tile_iter;
         } else {
-          uint16_t* yout = static_cast<uint16_t*>(p.out);
           const float gw = row_ok ? p.row_gate[row] : 0.0f;
           if (ok && row_ok && col_ok) {
-            uint4* dst = reinterpret_cast<uint4*>(yout + row * p.N + it.n * 256 + hf * 128);
+            uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.out) + row * p.N + col0);
 #pragma unroll
             for (int w = 0; w < 16; ++w) {
               const float2 a0 = acc[4 * w], a1 = acc[4 * w + 1], a2 = acc[4 * w + 2], a3 = acc[4 * w + 3];
@@ -399,40 +514,63 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   tc_fence_before_sync();
   __syncthreads();
+  if (kPair) cluster_sync();  // neither CTA frees the pair's TMEM while the other still reads it
   if (warp == 1) {
     tc_fence_after_sync();
-    tmem_dealloc(tmem, 512);
+    if (kPair) tmem_dealloc_pair(tmem, 512);
+    else tmem_dealloc(tmem, 512);
   }
 }
 
-template <bool kFP8, bool kGemm1>
+template <bool kFP8, bool kGemm1, bool kPair>
 cudaError_t launch_one(const GemmParams& p, int grid, const CUtensorMap& a, const CUtensorMap& b0,
                        const CUtensorMap& b1, const CUtensorMap& bs0, const CUtensorMap& bs1, cudaStream_t s) {
-  auto kern = grouped_gemm_kernel<kFP8, kGemm1>;
+  auto kern = grouped_gemm_kernel<kFP8, kGemm1, kPair>;
   static bool attr_set = false;  // per process; one device's limit serves every B200
   if (!attr_set) {
     cudaError_t e =
-        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SmemLayout::kDynamic);
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Cfg<kPair>::kDynamic);
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  kern<<<grid, kThreads, SmemLayout::kDynamic, s>>>(p, a, b0, b1, bs0, bs1);
-  return cudaGetLastError();
+  if (!kPair) {
+    kern<<<grid, kThreads, Cfg<kPair>::kDynamic, s>>>(p, a, b0, b1, bs0, bs1);
+    return cudaGetLastError();
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(grid & ~1));
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = Cfg<kPair>::kDynamic;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, p, a, b0, b1, bs0, bs1);
 }
 
 }  // namespace
 
-cudaError_t launch_gemm1(const GemmParams& p, bool fp8, int grid, const CUtensorMap& tm_a, const CUtensorMap& tm_w1,
-                         const CUtensorMap& tm_w3, const CUtensorMap& tm_sw1, const CUtensorMap& tm_sw3,
-                         cudaStream_t s) {
-  return fp8 ? launch_one<true, true>(p, grid, tm_a, tm_w1, tm_w3, tm_sw1, tm_sw3, s)
-             : launch_one<false, true>(p, grid, tm_a, tm_w1, tm_w3, tm_sw1, tm_sw3, s);
+cudaError_t launch_gemm1(const GemmParams& p, bool fp8, bool pair, int grid, const CUtensorMap& tm_a,
+                         const CUtensorMap& tm_w1, const CUtensorMap& tm_w3, const CUtensorMap& tm_sw1,
+                         const CUtensorMap& tm_sw3, cudaStream_t s) {
+  if (pair)
+    return fp8 ? launch_one<true, true, true>(p, grid, tm_a, tm_w1, tm_w3, tm_sw1, tm_sw3, s)
+               : launch_one<false, true, true>(p, grid, tm_a, tm_w1, tm_w3, tm_sw1, tm_sw3, s);
+  return fp8 ? launch_one<true, true, false>(p, grid, tm_a, tm_w1, tm_w3, tm_sw1, tm_sw3, s)
+             : launch_one<false, true, false>(p, grid, tm_a, tm_w1, tm_w3, tm_sw1, tm_sw3, s);
 }
 
-cudaError_t launch_gemm2(const GemmParams& p, bool fp8, int grid, const CUtensorMap& tm_a, const CUtensorMap& tm_w2,
-                         const CUtensorMap& tm_sw2, cudaStream_t s) {
-  return fp8 ? launch_one<true, false>(p, grid, tm_a, tm_w2, tm_w2, tm_sw2, tm_sw2, s)
-             : launch_one<false, false>(p, grid, tm_a, tm_w2, tm_w2, tm_sw2, tm_sw2, s);
+cudaError_t launch_gemm2(const GemmParams& p, bool fp8, bool pair, int grid, const CUtensorMap& tm_a,
+                         const CUtensorMap& tm_w2, const CUtensorMap& tm_sw2, cudaStream_t s) {
+  if (pair)
+    return fp8 ? launch_one<true, false, true>(p, grid, tm_a, tm_w2, tm_w2, tm_sw2, tm_sw2, s)
+               : launch_one<false, false, true>(p, grid, tm_a, tm_w2, tm_w2, tm_sw2, tm_sw2, s);
+  return fp8 ? launch_one<true, false, false>(p, grid, tm_a, tm_w2, tm_w2, tm_sw2, tm_sw2, s)
+             : launch_one<false, false, false>(p, grid, tm_a, tm_w2, tm_w2, tm_sw2, tm_sw2, s);
 }
 
 }  // namespace moe

@@ -10,8 +10,9 @@
 //   1. histogram: one CTA per 256-token chunk counts its (token, slot) pairs
 //      per expert in shared memory -> chunk_base[e][chunk].
 //   2. scan: one CTA scans chunk counts per expert (one warp per expert), then
-//      the expert totals -> counts, offsets, and the per-group M-tile prefix
-//      the grouped GEMMs schedule from; chunk_base becomes absolute row bases.
+//      the expert totals -> counts, offsets, and the per-group prefixes of
+//      128-row tiles and 256-row pair tiles the grouped GEMMs schedule from;
+//      chunk_base becomes absolute row bases.
 //   3. scatter: each warp ranks its 32 tokens' pairs in (token, slot) order
 //      with __match_any_sync (equal experts in one 32-pair round rank by lane),
 //      warps are then offset by an exclusive scan over the CTA's 8 warps, and
@@ -71,25 +72,30 @@ __global__ void __launch_bounds__(1024) scan_kernel(const PermuteParams p) {
   __syncthreads();
   // offsets and M-tile prefix over the G groups
   if (warp == 0) {
-    int run_off = 0, run_mt = 0;
+    int run_off = 0, run_mt = 0, run_mp = 0;
     for (int g0 = 0; g0 < p.G; g0 += 32) {
       const int g = g0 + lane;
       const int c = g < p.G ? cnt_s[g] : 0;
       const int mt = (c + kTileM - 1) / kTileM;
+      const int mp = (c + 2 * kTileM - 1) / (2 * kTileM);
       const int ic = warp_inclusive_scan(c, lane);
       const int im = warp_inclusive_scan(mt, lane);
+      const int ip = warp_inclusive_scan(mp, lane);
       if (g < p.G) {
         p.counts[g] = c;
         p.offsets[g] = run_off + ic - c;
         p.mt_prefix[g] = run_mt + im - mt;
+        p.mp_prefix[g] = run_mp + ip - mp;
         off_s[g] = run_off + ic - c;
       }
       run_off += __shfl_sync(0xffffffffu, ic, 31);
       run_mt += __shfl_sync(0xffffffffu, im, 31);
+      run_mp += __shfl_sync(0xffffffffu, ip, 31);
     }
     if (lane == 0) {
       p.offsets[p.G] = run_off;
       p.mt_prefix[p.G] = run_mt;
+      p.mp_prefix[p.G] = run_mp;
     }
   }
   __syncthreads();

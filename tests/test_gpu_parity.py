@@ -249,8 +249,16 @@ def _expert_cases():
     ]
 
 
+@pytest.fixture(params=["single", "pair"])
+def variant(request, m):
+    """Run the test under each expert-GEMM variant (same result expected)."""
+    m.moe_set_gemm_variant(m.MOE_GEMM_SINGLE if request.param == "single" else m.MOE_GEMM_PAIR)
+    yield request.param
+    m.moe_set_gemm_variant(m.MOE_GEMM_AUTO)
+
+
 @pytest.mark.parametrize("shape", _expert_cases(), ids=lambda s: s.name)
-def test_experts_parity(m, shape):
+def test_experts_parity(m, shape, variant):
     import torch
     x, w = _inputs(shape)
     idx_r, gate_r, _ = oracle.route(x, w["router_w"], w["router_bias"], shape.top_k)
@@ -298,6 +306,7 @@ def _layer_cases():
 
 @pytest.mark.parametrize("shape,n_sample", _layer_cases(), ids=lambda v: getattr(v, "name", str(v)))
 def test_forward_parity(m, shape, n_sample):
+    """The automatic variant choice (pair GEMMs at T = 8192 and 32768, single below)."""
     x = synth.make_x(shape)
     w = synth.make_weights(shape)
     idx_r, gate_r, logits_r = oracle.route(x, w["router_w"], w["router_bias"], shape.top_k, want_logits=True)
@@ -314,6 +323,39 @@ def test_forward_parity(m, shape, n_sample):
     err = frob_rel(bf16_bits_to_f64(out[toks]), ref)
     assert err < tol_for(shape.wdtype), err
     assert np.all(np.isfinite(bf16_bits_to_f64(out)))
+
+
+@pytest.mark.parametrize("shape", [
+    synth.MoeShape("pair-big-groups-fp8", T=600, hidden=512, n_experts=8, top_k=2, n_shared=1, inter=256,
+                   wdtype=synth.WDTYPE_FP8, seed=20),
+    synth.MoeShape("pair-big-groups-bf16", T=600, hidden=512, n_experts=8, top_k=2, n_shared=1, inter=256,
+                   wdtype=synth.WDTYPE_BF16, seed=21),
+    synth.MoeShape("pair-odd-H-fp8", T=333, hidden=384, n_experts=6, top_k=2, n_shared=0, inter=384,
+                   wdtype=synth.WDTYPE_FP8, seed=22),
+], ids=lambda s: s.name)
+def test_forward_parity_both_variants(m, shape, variant):
+    """Groups of several hundred rows: several 256-row pair tiles and ragged ends."""
+    x, w = _inputs(shape)
+    idx_r, gate_r, logits_r = oracle.route(x, w["router_w"], w["router_bias"], shape.top_k, want_logits=True)
+    out, idx, gate = _forward(m, shape, x, m.upload_weights(w))
+    check_routing(idx, gate, logits_r, idx_r, gate_r)
+    toks = np.flatnonzero(unique_tokens(logits_r, shape.top_k))
+    ref, _, _ = oracle.moe_tokens(shape, w, x, idx_r, gate_r, tokens=toks)
+    err = frob_rel(bf16_bits_to_f64(out[toks]), ref)
+    assert err < tol_for(shape.wdtype), err
+
+
+def test_variants_agree_bit_for_bit_on_bf16(m):
+    """Both GEMM variants accumulate each K stage in the same order in fp32 TMEM."""
+    shape = synth.MoeShape("agree", T=400, hidden=512, n_experts=6, top_k=2, n_shared=1, inter=256, seed=23)
+    x, w = _inputs(shape)
+    wd = m.upload_weights(w)
+    outs = []
+    for v in (m.MOE_GEMM_SINGLE, m.MOE_GEMM_PAIR):
+        m.moe_set_gemm_variant(v)
+        outs.append(_forward(m, shape, x, wd)[0])
+    m.moe_set_gemm_variant(m.MOE_GEMM_AUTO)
+    assert frob_rel(bf16_bits_to_f64(outs[0]), bf16_bits_to_f64(outs[1])) < 1e-3
 
 
 def test_forward_zero_tokens_is_a_noop(m):
