@@ -18,6 +18,9 @@ constexpr int kRouterTargetCtas = 148;
 
 // The 2-SM (CTA pair) expert GEMMs pay off once expert groups average more
 // than this many rows (below it, the pair's second half is mostly padding).
+// AUTO uses them for BF16 experts only: with FP8 experts every 128-deep K block
+// needs a TMEM hand-off between the MMA and both SMs' epilogues, and the
+// cross-SM round trip then limits the pair below the single-CTA kernel.
 constexpr int64_t kPairMinRowsPerGroup = 100;
 int g_gemm_variant = MOE_GEMM_AUTO;
 
@@ -222,7 +225,7 @@ int run_experts(const moe_config* c, const WsLayout& L, int64_t T, const void* x
   const int sms = sm_count();
   if (sms <= 0) return MOE_ERR_CUDA;
   const bool pair = g_gemm_variant == MOE_GEMM_PAIR ||
-                    (g_gemm_variant == MOE_GEMM_AUTO && R >= kPairMinRowsPerGroup * (E + S));
+                    (g_gemm_variant == MOE_GEMM_AUTO && !fp8 && R >= kPairMinRowsPerGroup * (E + S));
 
   GatherParams gp{};
   gp.T = (int32_t)T;
@@ -335,7 +338,7 @@ WsLayout ws_layout(const moe_config& c, int64_t T, int target_ctas) {
     off = (size_t)round_up((int64_t)(off + (bytes ? bytes : 1)), 1024);
     return o;
   };
-  L.status = take(256);
+  L.status = take(16384);  // status word, first-timeout record, debug counters
   L.idx = take((size_t)T * k * 4);
   L.gate = take((size_t)T * k * 4);
   L.logits_part = take((size_t)L.ksplit * T * E * 4);
@@ -385,7 +388,7 @@ int moe_forward(const moe_config* cfg, int64_t T, const void* x, const moe_weigh
   if (T == 0) return MOE_OK;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
-  CUDA_TRY(cudaMemsetAsync(ws + L.status, 0, 256, s));
+  CUDA_TRY(cudaMemsetAsync(ws + L.status, 0, 16384, s));
   Prof prof(s);
   int32_t* idx = topk_idx ? topk_idx : reinterpret_cast<int32_t*>(ws + L.idx);
   float* gate = topk_w ? topk_w : reinterpret_cast<float*>(ws + L.gate);
@@ -427,7 +430,7 @@ int moe_route(const moe_config* cfg, int64_t T, const void* x, const void* route
   if (T == 0) return MOE_OK;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
-  CUDA_TRY(cudaMemsetAsync(ws + L.status, 0, 256, s));
+  CUDA_TRY(cudaMemsetAsync(ws + L.status, 0, 16384, s));
   Prof prof(s);
   prof.on = false;
   return run_route(cfg, L, T, x, router_w, router_bias, topk_idx, topk_w, logits, ws, s, prof);
@@ -461,7 +464,7 @@ int moe_permute(const moe_config* cfg, int64_t T, const int32_t* topk_idx, int32
   if ((rc = check_ws(cfg, T, workspace, workspace_bytes, &L)) != MOE_OK) return rc;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
-  CUDA_TRY(cudaMemsetAsync(ws + L.status, 0, 256, s));
+  CUDA_TRY(cudaMemsetAsync(ws + L.status, 0, 16384, s));
   if (T == 0) {
     const int G = cfg->n_experts + cfg->n_shared;
     CUDA_TRY(cudaMemsetAsync(counts, 0, (size_t)G * 4, s));
@@ -491,7 +494,7 @@ int moe_experts(const moe_config* cfg, int64_t T, const void* x, const int32_t* 
   if (T == 0) return MOE_OK;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
-  CUDA_TRY(cudaMemsetAsync(ws + L.status, 0, 256, s));
+  CUDA_TRY(cudaMemsetAsync(ws + L.status, 0, 16384, s));
   Prof prof(s);
   prof.on = false;
   PermuteParams pp = permute_params(cfg, L, T, topk_idx, topk_w, ws);

@@ -73,13 +73,16 @@ struct Cfg {
   static constexpr int kTileRows = kPair ? 2 * kTileM : kTileM;      // rows of one work item
   static constexpr size_t kTiles = (size_t)kStages * kStageBytes;
   static constexpr size_t kScales = kTiles;                           // float [kScRing][kScSlot]
-  static constexpr size_t kBars = kScales + kScRing * kScSlot * 4;    // 2 kMaxStages + 5 + 2 kScRing barriers
-  static constexpr size_t kMisc = kBars + 256;                        // tmem slot, abort flag
+  static constexpr size_t kBars = kScales + kScRing * kScSlot * 4;    // mbarriers (kNumBars x 8 bytes)
+  static constexpr int kNumBars = 2 * kMaxStages + 2 + 2 + 1 + 2 * kScRing;
+  static constexpr size_t kMisc = kBars + ((kNumBars * 8 + 127) / 128) * 128;  // tmem slot, abort flag
   static constexpr size_t kAmax = kMisc + 64;                         // float [2][2][128]
   static constexpr size_t kMt = kAmax + 2 * 2 * 128 * 4;              // int [kMaxGroups + 1]
   static constexpr size_t kOff = kMt + (kMaxGroups + 1) * 4;          // int [kMaxGroups + 1]
   static constexpr size_t kEnd = kOff + (kMaxGroups + 1) * 4;
   static constexpr size_t kDynamic = kEnd + 1024;                     // + alignment slack
+  static_assert(kMisc >= kBars + kNumBars * 8, "mbarriers overlap the misc words");
+  static_assert(kDynamic <= 227 * 1024, "shared memory budget");
 };
 
 struct Item {
@@ -131,9 +134,10 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
 // Bounded wait by every lane, with a warp-uniform verdict (keeps the warp
 // converged for the .sync.aligned TMEM loads that follow).
 template <bool kCluster>
-__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, int* status, volatile int* abort_flag) {
-  const bool ok = kCluster ? mbar_wait_cluster(bar, parity, status, abort_flag)
-                           : mbar_wait(bar, parity, status, abort_flag);
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, int* status, volatile int* abort_flag,
+                                          int site, int progress) {
+  const bool ok = kCluster ? mbar_wait_cluster(bar, parity, status, abort_flag, site, progress)
+                           : mbar_wait(bar, parity, status, abort_flag, site, progress);
   return __all_sync(0xffffffffu, ok);
 }
 
@@ -180,11 +184,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&tfull[b], 1);
-      mbar_init(&tempty[b], kPair ? 2 * kEpiThreads : kEpiThreads);
+      mbar_init(&tempty[b], kPair ? 2 * kEpiWarps : kEpiWarps);  // one arrival per epilogue warp
     }
     for (int j = 0; j < kScRing; ++j) {
       mbar_init(&scfull[j], 32);
-      mbar_init(&scempty[j], kEpiThreads);
+      mbar_init(&scempty[j], kEpiWarps);
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -216,6 +220,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int kstages = p.K / kElemsPerStage;
   const int nkb = p.K / 128;
   const int my_off = kPair ? kTileM * (int)rank : 0;  // this CTA's rows inside a work item
+  // Wait-site codes recorded with a timeout: kernel variant, CTA rank, wait.
+  const int site0 = (kFP8 ? 0x100 : 0) | (kGemm1 ? 0x200 : 0) | (kPair ? 0x400 : 0) | (int)(rank << 11);
+#ifdef MOE_DEBUG_STATE
+  int dbg_a = -1, dbg_b = -1, dbg_c = -1;
+#define MOE_DBG(a, b, c) (dbg_a = (int)(a), dbg_b = (int)(b), dbg_c = (int)(c))
+#else
+#define MOE_DBG(a, b, c) ((void)0)
+#endif
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer --
@@ -247,7 +259,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       for (int ks = 0; ks < kstages; ++ks) {
         bool w = true;
-        if (lane == 0) w = mbar_wait(&empty[stage], phase ^ 1, p.status, abort_flag);
+        MOE_DBG(item, ks, sc_iter);
+        if (lane == 0) w = mbar_wait(&empty[stage], phase ^ 1, p.status, abort_flag, site0 | 1, item);
         if (!__shfl_sync(0xffffffffu, w ? 1 : 0, 0)) { ok = false; break; }
         if (lane == 0) {
           const int kx = ks * kElemsPerStage;
@@ -268,7 +281,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (kFP8) {
           const uint32_t j = sc_iter % kScRing, sph = (sc_iter / kScRing) & 1u;
-          if (!warp_wait<false>(&scempty[j], sph ^ 1u, p.status, abort_flag)) { ok = false; break; }
+          if (!warp_wait<false>(&scempty[j], sph ^ 1u, p.status, abort_flag, site0 | 2, item)) { ok = false; break; }
           float* slot = sc + j * kScSlot;
           const float* src = p.a_scale + (int64_t)ks * p.rows_pad + my_row0 + lane * 4;
 #pragma unroll
@@ -308,9 +321,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (kPair) mma_commit_pair(bar, 0x3);
         else mma_commit(bar);
       };
-      auto wait_tempty = [&](uint32_t b, uint32_t par) {
-        return kPair ? mbar_wait_cluster(&tempty[b], par, p.status, abort_flag)
-                     : mbar_wait(&tempty[b], par, p.status, abort_flag);
+      auto wait_tempty = [&](uint32_t b, uint32_t par, uint32_t it) {
+        return kPair ? mbar_wait_cluster(&tempty[b], par, p.status, abort_flag, site0 | 3, (int)it)
+                     : mbar_wait(&tempty[b], par, p.status, abort_flag, site0 | 3, (int)it);
       };
       int stage = 0;
       uint32_t phase = 0;
@@ -319,11 +332,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int item = unit; item < total && ok; item += n_units) {
         if (!kFP8) {
           const uint32_t b = acc_iter & 1u, tph = (acc_iter >> 1) & 1u;
-          if (!wait_tempty(b, tph ^ 1u)) { ok = false; break; }
+          if (!wait_tempty(b, tph ^ 1u, acc_iter)) { ok = false; break; }
           tc_fence_after_sync();
           const uint32_t d = tmem + b * 256;
           for (int ks = 0; ks < kstages; ++ks) {
-            if (!mbar_wait(&full[stage], phase, p.status, abort_flag)) { ok = false; break; }
+            if (!mbar_wait(&full[stage], phase, p.status, abort_flag, site0 | 4, (int)acc_iter)) { ok = false; break; }
             tc_fence_after_sync();
             const uint64_t ad = sdesc_k_sw128(sA + stage * kABytes);
             const uint64_t bd = sdesc_k_sw128(sB + stage * C::kBBytes);
@@ -338,8 +351,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         } else {
           for (int ks = 0; ks < kstages; ++ks) {
             const uint32_t b = acc_iter & 1u, tph = (acc_iter >> 1) & 1u;
-            if (!wait_tempty(b, tph ^ 1u)) { ok = false; break; }
-            if (!mbar_wait(&full[stage], phase, p.status, abort_flag)) { ok = false; break; }
+            MOE_DBG(item, ks, acc_iter);
+            if (!wait_tempty(b, tph ^ 1u, acc_iter)) { ok = false; break; }
+            if (!mbar_wait(&full[stage], phase, p.status, abort_flag, site0 | 4, (int)acc_iter)) { ok = false; break; }
             tc_fence_after_sync();
             const uint32_t d = tmem + b * 256;
             const uint64_t ad = sdesc_k_sw128(sA + stage * kABytes);
@@ -368,8 +382,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     // The accumulator is released on the pair's even CTA (or locally).
     auto release_acc = [&](uint32_t b) {
       tc_fence_before_sync();
-      if (kPair) mbar_arrive_cluster(map_to_cta(&tempty[b], 0));
-      else mbar_arrive(&tempty[b]);
+      __syncwarp();
+      if (lane == 0) {
+        if (kPair) mbar_arrive_cluster(map_to_cta(&tempty[b], 0));
+        else mbar_arrive(&tempty[b]);
+      }
     };
     uint32_t acc_iter = 0, tile_iter = 0, sc_iter = 0;
     bool ok = true;
@@ -383,7 +400,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool col_ok = col0 < p.N;
       if (!kFP8) {
         const uint32_t b = acc_iter & 1u, tph = (acc_iter >> 1) & 1u;
-        if (ok) ok = warp_wait<kPair>(&tfull[b], tph, p.status, abort_flag);
+        if (ok) ok = warp_wait<false>(&tfull[b], tph, p.status, abort_flag, site0 | 6, (int)acc_iter);
         tc_fence_after_sync();
         const uint32_t base = tmem + lane_base + b * 256;
         if (kGemm1) {
@@ -432,18 +449,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int i = 0; i < 64; ++i) acc[i] = make_float2(0.0f, 0.0f);
         for (int kb = 0; kb < nkb; ++kb) {
           const uint32_t j = sc_iter % kScRing, sph = (sc_iter / kScRing) & 1u;
-          if (ok) ok = warp_wait<false>(&scfull[j], sph, p.status, abort_flag);
+          MOE_DBG(item, kb, acc_iter);
+          if (ok) ok = warp_wait<false>(&scfull[j], sph, p.status, abort_flag, site0 | 5, (int)sc_iter);
           const float* slot = sc + j * kScSlot;
           const float a_s = slot[rl];
           const float s0 = slot[128], s1 = slot[129];
-          mbar_arrive(&scempty[j]);
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&scempty[j]);
           ++sc_iter;
           // GEMM1: the first 64 columns are gate columns (s0), the next 64 up columns (s1).
           // GEMM2: the half's 128 columns sit in n-block 2n (hf 0, s0) or 2n+1 (s1).
           const float f0 = a_s * ((kGemm1 || hf == 0) ? s0 : s1);
           const float f1 = kGemm1 ? a_s * s1 : f0;
           const uint32_t b = acc_iter & 1u, tph = (acc_iter >> 1) & 1u;
-          if (ok) ok = warp_wait<kPair>(&tfull[b], tph, p.status, abort_flag);
+          if (ok) ok = warp_wait<false>(&tfull[b], tph, p.status, abort_flag, site0 | 6, (int)acc_iter);
           tc_fence_after_sync();
           const uint32_t base = tmem + lane_base + b * 256;
           constexpr int kNch = 128 / kFp8Chunk;  // chunks per thread per K block
@@ -512,6 +531,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   }
+#ifdef MOE_DEBUG_STATE
+  // Debug builds: each role's final counters, 16 ints per block from status[64].
+  if (kGemm1 && lane == 0 && blockIdx.x < 900) {
+    int* dbg = p.status + 64 + blockIdx.x * 16;
+    if (warp == 0) { dbg[0] = dbg_a; dbg[1] = dbg_b; dbg[2] = dbg_c; }
+    if (warp == 1) { dbg[3] = dbg_a; dbg[4] = dbg_b; dbg[5] = dbg_c; }
+    if (warp == 2) { dbg[6] = dbg_a; dbg[7] = dbg_b; dbg[8] = dbg_c; }
+    if (warp == 6) { dbg[9] = dbg_a; dbg[10] = dbg_b; dbg[11] = dbg_c; }
+    if (warp == 0) dbg[12] = total;
+  }
+#endif
   tc_fence_before_sync();
   __syncthreads();
   if (kPair) cluster_sync();  // neither CTA frees the pair's TMEM while the other still reads it

@@ -29,6 +29,16 @@ __device__ __forceinline__ void latch_status(int* status, int code) {
   if (status) atomicCAS(status, 0, code);
 }
 
+// Latch a timeout and, for the first one only, where it happened: status[1] =
+// wait site, status[2] = block index, status[3] = the site's progress counter.
+__device__ __forceinline__ void latch_timeout(int* status, int site, int progress) {
+  if (status && atomicCAS(status, 0, MOE_ERR_DEVICE_TIMEOUT) == 0) {
+    status[1] = site;
+    status[2] = (int)blockIdx.x;
+    status[3] = progress;
+  }
+}
+
 // ---------------------------------------------------------------- mbarrier --
 
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
@@ -64,7 +74,7 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 // false (and latches a timeout, and raises the CTA's abort flag) if it does not
 // complete within kWaitLimitNs, or if another role of the CTA already aborted.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* status,
-                                          volatile int* abort_flag) {
+                                          volatile int* abort_flag, int site = 0, int progress = 0) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
   uint32_t spins = 0;
@@ -73,7 +83,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* s
     if ((++spins & 63u) == 0) {
       if (*abort_flag) return false;
       if (global_timer_ns() - t0 > kWaitLimitNs) {
-        latch_status(status, MOE_ERR_DEVICE_TIMEOUT);
+        latch_timeout(status, site, progress);
         *abort_flag = 1;
         return false;
       }
@@ -178,7 +188,7 @@ __device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t pa
 
 // Bounded wait with cluster-scope acquire (for barriers that peer CTAs arrive on).
 __device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity, int* status,
-                                                  volatile int* abort_flag) {
+                                                  volatile int* abort_flag, int site = 0, int progress = 0) {
   if (mbar_try_wait_cluster(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
   uint32_t spins = 0;
@@ -187,7 +197,7 @@ __device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity
     if ((++spins & 63u) == 0) {
       if (*abort_flag) return false;
       if (global_timer_ns() - t0 > kWaitLimitNs) {
-        latch_status(status, MOE_ERR_DEVICE_TIMEOUT);
+        latch_timeout(status, site, progress);
         *abort_flag = 1;
         return false;
       }
