@@ -156,6 +156,29 @@ MOE_API int moe_permute(const moe_config* cfg, int64_t T, const int32_t* topk_id
                 int32_t* offsets, int32_t* perm, int32_t* pos, void* workspace, size_t workspace_bytes,
                 moe_stream_t stream);
 
+/* moe_permute without a workspace, for callers that cannot allocate device
+ * memory: a plugin whose host framework owns all device memory, a serving loop
+ * that reserved its memory up front, or a latency-critical path that cannot
+ * afford an allocation. The pages describe no such entry point; it is a
+ * property of this library, not of the layer.
+ * Same inputs, outputs and results as moe_permute. Its scratch is a fixed
+ * 1 MiB device array inside the library (every GPU that loads the library
+ * holds it until the process exits), so E * ceil(T / 256) must not exceed
+ * 260,032 (T <= 188,928 tokens at E = 352); larger sizes return
+ * MOE_ERR_UNSUPPORTED_SHAPE without touching the device.
+ * device_status (optional, device memory, one int) receives the device status
+ * (MOE_ERR_BAD_INDEX for skipped pairs); the call zeroes it first. Without it
+ * the status word lives in the shared scratch.
+ * The first call with a given device current looks up the scratch address on
+ * that device; make that first call before any stream capture. Every call
+ * shares the one scratch array per device: calls whose work overlaps on the
+ * GPU (other streams, other threads) race and must be serialised by the
+ * caller. The call allocates nothing: no cudaMalloc, cudaFree or allocating
+ * library routine. */
+MOE_API int moe_permute_noalloc(const moe_config* cfg, int64_t T, const int32_t* topk_idx, int32_t* counts,
+                                int32_t* offsets, int32_t* perm, int32_t* pos, int* device_status,
+                                moe_stream_t stream);
+
 /* Expert MLPs for a given routing: permute, gather (+ quantise), gate/up GEMM
  * with SwiGLU, down GEMM. y [(k+S)T, H] bf16 receives each row's expert output
  * times its gate (1 for shared rows); pos [T, k+S] receives the row of each

@@ -9,7 +9,7 @@ The functions carry the names of the C entry points:
   moe_workspace_bytes, moe_forward, moe_forward_host, moe_route,
   moe_quantize_act, moe_permute, moe_experts, moe_combine, moe_read_status,
   moe_status_string, moe_profile_enable, moe_profile_read, moe_device_sm_count,
-  moe_set_gemm_variant.
+  moe_set_gemm_variant, moe_permute_noalloc.
 """
 from __future__ import annotations
 
@@ -79,6 +79,7 @@ def load():
         "moe_profile_kernel_name": [ctypes.c_int],
         "moe_device_sm_count": [ctypes.POINTER(ctypes.c_int)],
         "moe_set_gemm_variant": [ctypes.c_int],
+        "moe_permute_noalloc": [cfgp, i64, vp, vp, vp, vp, vp, vp, vp],
     }
     for name, args in sig.items():
         f = getattr(lib, name)
@@ -158,6 +159,13 @@ def moe_permute(cfg, T, topk_idx, counts, offsets, perm, pos, workspace, stream=
     nb = workspace.numel() * workspace.element_size()
     _check(load().moe_permute(ctypes.byref(cfg), T, _ptr(topk_idx), _ptr(counts), _ptr(offsets), _ptr(perm),
                               _ptr(pos), _ptr(workspace), nb, _stream(stream)), "moe_permute")
+
+
+def moe_permute_noalloc(cfg, T, topk_idx, counts, offsets, perm, pos, device_status=None, stream=None):
+    """moe_permute without a workspace (fixed static scratch inside the library)."""
+    _check(load().moe_permute_noalloc(ctypes.byref(cfg), T, _ptr(topk_idx), _ptr(counts), _ptr(offsets),
+                                      _ptr(perm), _ptr(pos), _ptr(device_status), _stream(stream)),
+           "moe_permute_noalloc")
 
 
 def moe_experts(cfg, T, x, topk_idx, topk_w, w: moe_weights, y, pos, workspace, stream=None):
