@@ -178,7 +178,7 @@ def run_ours(args):
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=f"cuda:{local}")
     stream = torch.cuda.current_stream()
 
-    def measure(T, x_host, e2e=True, profile=True):
+    def measure(T, x_host, e2e=True, profile=True, shape=shape, wts=wts):
         cfg = m.make_config(shape.hidden, shape.n_experts, shape.top_k, shape.n_shared, shape.inter, shape.wdtype)
         x = m.to_device(x_host, f"cuda:{local}")
         out = torch.empty((T, shape.hidden), dtype=torch.bfloat16, device=f"cuda:{local}")
@@ -251,9 +251,20 @@ def run_ours(args):
         if not args.no_decode and shape.wdtype == synth.WDTYPE_FP8 and shape.T != 64:
             dshape = shape.with_tokens(64)
             decode = measure(64, synth.make_x(dshape), e2e=False)
+    decode_bf16 = None
+    if not args.no_decode and shape.wdtype == synth.WDTYPE_FP8:
+        # The BF16 decode workload (its own seed and BF16 weights).
+        del wd, wts
+        torch.cuda.empty_cache()
+        bshape = synth.DECODE_BF16
+        bw = m.upload_weights(synth.make_weights(bshape), f"cuda:{local}")
+        with ClockSampler(local):
+            decode_bf16 = (bshape, measure(bshape.T, synth.make_x(bshape), e2e=False, shape=bshape,
+                                           wts=m.make_weights(bw)))
+        del bw
     clocks = clk.summary()
 
-    def roofline(res, T):
+    def roofline(res, T, shape=shape):
         """The dominant kernel against its bound (HBM bytes or tensor FLOPs)."""
         idx = res["idx"]
         touched = int(np.unique(idx).size)
@@ -314,6 +325,14 @@ def run_ours(args):
                               "layer_roofline": dlayer,
                               "kernel_ms": {k: round(v, 4) for k, v in decode["kernel_ms"].items()},
                               "config": "T=64, same layer and weights as the headline workload"}
+    if decode_bf16 is not None:
+        bshape, bres = decode_bf16
+        broof, blayer = roofline(bres, bshape.T, shape=bshape)
+        line["decode_bf16_t64"] = {"value": round(bres["tokens_per_s"], 1), "unit": "tokens/s",
+                                   "ms_per_step": round(bres["ms_per_step"], 4), "roofline": broof,
+                                   "layer_roofline": blayer,
+                                   "kernel_ms": {k: round(v, 4) for k, v in bres["kernel_ms"].items()},
+                                   "config": describe(bshape)}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(shape, x_np, w_np)
     if rank == 0:

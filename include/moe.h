@@ -213,10 +213,9 @@ MOE_API int moe_profile_read(float* ms, int n, int* n_out);
 MOE_API const char* moe_profile_kernel_name(int i);
 
 /* Expert-GEMM variant (process-wide; default MOE_GEMM_AUTO). SINGLE runs one
- * CTA per 128-row tile; PAIR runs 2-SM CTA pairs on 256-row tiles (less L2
- * traffic per FLOP when expert groups are large); AUTO picks PAIR for BF16
- * experts when groups average at least 100 rows, SINGLE otherwise. All
- * variants compute the same result. */
+ * CTA per 128-row tile; PAIR runs 2-SM CTA pairs on 256-row tiles (each weight
+ * tile crosses L2 -> SM once per 256 rows). AUTO currently runs SINGLE, the
+ * faster of the two for FP8 experts. All variants compute the same result. */
 enum { MOE_GEMM_AUTO = 0, MOE_GEMM_SINGLE = 1, MOE_GEMM_PAIR = 2 };
 MOE_API int moe_set_gemm_variant(int variant);
 

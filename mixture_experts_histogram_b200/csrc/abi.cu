@@ -16,12 +16,10 @@ namespace {
 // CTAs the router aims for when it splits K for small token counts (B200: 148 SMs).
 constexpr int kRouterTargetCtas = 148;
 
-// The 2-SM (CTA pair) expert GEMMs pay off once expert groups average more
-// than this many rows (below it, the pair's second half is mostly padding).
-// AUTO uses them for BF16 experts only: with FP8 experts every 128-deep K block
-// needs a TMEM hand-off between the MMA and both SMs' epilogues, and the
-// cross-SM round trip then limits the pair below the single-CTA kernel.
-constexpr int64_t kPairMinRowsPerGroup = 100;
+// Expert-GEMM variant. AUTO runs the single-CTA kernels: with FP8 experts the
+// 2-SM pair needs a TMEM hand-off between the MMA and both SMs' epilogues for
+// every 128-deep K block, and that cross-SM round trip made it slower than
+// the single-CTA kernel at T = 8192 (2.72 vs 1.56 ms for the gate/up GEMM).
 int g_gemm_variant = MOE_GEMM_AUTO;
 
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
@@ -224,8 +222,7 @@ int run_experts(const moe_config* c, const WsLayout& L, int64_t T, const void* x
   const int64_t R = L.R;
   const int sms = sm_count();
   if (sms <= 0) return MOE_ERR_CUDA;
-  const bool pair = g_gemm_variant == MOE_GEMM_PAIR ||
-                    (g_gemm_variant == MOE_GEMM_AUTO && !fp8 && R >= kPairMinRowsPerGroup * (E + S));
+  const bool pair = g_gemm_variant == MOE_GEMM_PAIR;
 
   GatherParams gp{};
   gp.T = (int32_t)T;
@@ -264,6 +261,7 @@ int run_experts(const moe_config* c, const WsLayout& L, int64_t T, const void* x
   g1.K = H;
   g1.N = I;
   g1.n_tiles = I / 128;
+  g1.n_fastest = 0;
   g1.R = (int32_t)R;
   g1.rows_pad = L.rows_pad;
   g1.a_scale = fp8 ? reinterpret_cast<const float*>(ws + L.sxp) : nullptr;
@@ -282,6 +280,7 @@ int run_experts(const moe_config* c, const WsLayout& L, int64_t T, const void* x
   g2.K = I;
   g2.N = H;
   g2.n_tiles = (int32_t)ceil_div(H, 256);
+  g2.n_fastest = 1;
   g2.a_scale = fp8 ? reinterpret_cast<const float*>(ws + L.sh) : nullptr;
   g2.b_scale0 = w->s2;
   g2.b_scale1 = w->s2;

@@ -84,6 +84,7 @@ struct GemmParams {
   int32_t G, E;              // groups, routed experts (group E is the shared expert)
   int32_t K, N;              // reduction length; output width (I for GEMM1, H for GEMM2)
   int32_t n_tiles;           // output tiles per M tile
+  int32_t n_fastest;         // item order: 1 = N tiles of a row tile adjacent, 0 = M tiles adjacent
   int32_t R;                 // total rows
   int64_t rows_pad;          // row stride of transposed activation scales
   const float* a_scale;      // FP8: [K/128, rows_pad]

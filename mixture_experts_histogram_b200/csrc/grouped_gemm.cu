@@ -26,9 +26,10 @@
 //     tile crosses L2 -> SM once per pair instead of once per 128 rows: a third
 //     less L2 traffic per FLOP, for groups with more than ~100 rows.
 //
-// Persistent CTAs (pairs) walk a static list of work items; an item is
-// (group, N tile, M tile) with the M tiles of one (group, N tile) adjacent, so
-// CTAs that share a weight tile run together and the second read hits L2.
+// Persistent CTAs (pairs) walk a static list of work items (group, N tile,
+// M tile). GEMM1 keeps the M tiles of one (group, N tile) adjacent, so CTAs
+// sharing a weight tile run together; GEMM2 keeps the N tiles of one row tile
+// adjacent (its h rows are re-read by 16 N tiles), which measured faster.
 // Warp roles:
 //   warp 0      producer. Lane 0 issues the TMA loads. In FP8 mode all 32 lanes
 //               also cp.async each K block's 128 row scales and two
@@ -65,6 +66,7 @@ constexpr int kScSlot = 132;                    // floats: 128 row scales + 2 bl
 #endif
 constexpr int kFp8Chunk = MOE_FP8_CHUNK;        // TMEM columns per load when promoting FP8 partials
 
+
 template <bool kPair>
 struct Cfg {
   static constexpr int kStages = kPair ? 6 : 4;
@@ -89,8 +91,10 @@ struct Item {
   int g, n, row0, end;  // group, N tile, first row of the tile, end of the group's rows
 };
 
+// n_fastest: consecutive items walk the N tiles of one row tile (they share A
+// rows); otherwise they walk the M tiles of one weight tile (they share B).
 __device__ __forceinline__ Item decode_item(int item, int n_tiles, int G, int tile_rows, const int* s_mt,
-                                            const int* s_off) {
+                                            const int* s_off, bool n_fastest) {
   const int q = item / n_tiles;
   int lo = 0, hi = G;  // s_mt[lo] <= q < s_mt[hi]
   while (hi - lo > 1) {
@@ -102,8 +106,8 @@ __device__ __forceinline__ Item decode_item(int item, int n_tiles, int G, int ti
   it.g = lo;
   const int mtiles = s_mt[lo + 1] - s_mt[lo];
   const int local = item - n_tiles * s_mt[lo];
-  it.n = local / mtiles;
-  it.row0 = s_off[lo] + (local % mtiles) * tile_rows;
+  it.n = n_fastest ? local % n_tiles : local / mtiles;
+  it.row0 = s_off[lo] + (n_fastest ? local / n_tiles : local % mtiles) * tile_rows;
   it.end = s_off[lo + 1];
   return it;
 }
@@ -237,7 +241,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t issued_phase = 0;  // bit s: the phase of that last issue
     bool ok = true;
     for (int item = unit; item < total && ok; item += n_units) {
-      const Item it = decode_item(item, p.n_tiles, p.G, C::kTileRows, s_mt, s_off);
+      const Item it = decode_item(item, p.n_tiles, p.G, C::kTileRows, s_mt, s_off, p.n_fastest != 0);
       const bool shared = (it.g == p.E);
       const int my_row0 = it.row0 + my_off;
       const BRows<kGemm1> rows(it, p, &tm_b0, &tm_b1, &tm_bs0, &tm_bs1);
@@ -391,7 +395,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t acc_iter = 0, tile_iter = 0, sc_iter = 0;
     bool ok = true;
     for (int item = unit; item < total; item += n_units) {
-      const Item it = decode_item(item, p.n_tiles, p.G, C::kTileRows, s_mt, s_off);
+      const Item it = decode_item(item, p.n_tiles, p.G, C::kTileRows, s_mt, s_off, p.n_fastest != 0);
       const int64_t row = (int64_t)it.row0 + my_off + rl;
       const bool row_ok = row < it.end;
       // Output columns of this thread: GEMM1 h columns n*128 + 64 hf (+64);
