@@ -147,6 +147,29 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm), "samples_under_load": len(loaded)}
 
 
+# ------------------------------------------------------------ replicas ----
+
+def max_over_ranks(value: float, world: int, device=None) -> float:
+    """The largest of every rank's value (device time of the same timed region).
+
+    Every rank calls this the same number of times, in the same order; with one
+    rank it returns `value` unchanged.
+    """
+    if world <= 1:
+        return float(value)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def replica_throughput(tokens_per_rank: int, world: int, steps: int, max_total_ms: float) -> float:
+    """Whole-job tokens/s of `world` independent replicas: all ranks' tokens over
+    the slowest rank's time for the same `steps`."""
+    return world * tokens_per_rank * steps / (max_total_ms / 1e3)
+
+
 # --------------------------------------------------------------- our arm ----
 
 def run_ours(args):
@@ -214,15 +237,11 @@ def run_ours(args):
         m.moe_profile_enable(False)
         if world > 1:
             dist.barrier()
-        total_ms = sum(a.elapsed_time(b) for a, b in ev)
-        t = torch.tensor([total_ms], dtype=torch.float64, device=f"cuda:{local}")
-        if world > 1:
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+        total_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in ev), world, f"cuda:{local}")
         st = m.moe_read_status(ws)
         if st != 0:
             raise RuntimeError(f"device status after timing: {m.moe_status_string(st)}")
-        res = {"ms_per_step": total_ms / args.steps, "tokens_per_s": world * T * args.steps / (total_ms / 1e3),
+        res = {"ms_per_step": total_ms / args.steps, "tokens_per_s": replica_throughput(T, world, args.steps, total_ms),
                "kernel_ms": {k: v / args.steps for k, v in per_kernel.items()},
                "idx": idx.cpu().numpy()}
         if e2e:
@@ -237,10 +256,8 @@ def run_ours(args):
                 t0 = time.perf_counter()
                 m.moe_forward_host(cfg, T, xh, wts, oh, ws, stream=stream)
                 ms.append((time.perf_counter() - t0) * 1e3)
-            tt = torch.tensor([sum(ms)], dtype=torch.float64, device=f"cuda:{local}")
-            if world > 1:
-                dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-            res["e2e"] = {"value": world * T * args.steps / (float(tt.item()) / 1e3), "unit": "tokens/s",
+            e2e_ms = max_over_ranks(sum(ms), world, f"cuda:{local}")
+            res["e2e"] = {"value": replica_throughput(T, world, args.steps, e2e_ms), "unit": "tokens/s",
                           "h2d_bytes_per_step": T * shape.hidden * 2, "d2h_bytes_per_step": T * shape.hidden * 2}
         return res
 
@@ -406,7 +423,7 @@ def run_reference(args):
         _oracle_sample(shape, x_np, w_np, n)
     ts = [_oracle_sample(shape, x_np, w_np, n) for _ in range(steps)]
     value = n * steps / sum(ts)
-    line = {"metric": METRIC, "value": round(value, 3), "unit": "tokens/s", "n_gpus": 0, "steps": steps,
+    line = {"metric": METRIC, "value": round(value, 3), "unit": "tokens/s", "n_gpus": args.gpus, "steps": steps,
             "warmup": warm, "ms_per_step": round(1e3 * sum(ts) / steps, 2), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64 accumulation (oracle)",
             "data": "synthetic (seeded, counter-based generator)", "impl": "reference",
