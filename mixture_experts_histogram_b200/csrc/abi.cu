@@ -124,7 +124,7 @@ struct Prof {
 };
 
 struct Maps {
-  CUtensorMap x, wr, xp, w1, w3, sw1, sw3, h, w2, sw2;
+  CUtensorMap x, wr, xp, w1, w3, sw1, sw3, h, w2, sw2, w2h, sw2h;  // w2h/sw2h: 128-row boxes
 };
 
 void router_shape(int E, int* nbox, int* box_rows) {
@@ -242,14 +242,16 @@ int run_experts(const moe_config* c, const WsLayout& L, int64_t T, const void* x
             map_2d(&m.w1, w->w1, fp8, H, (uint64_t)E * I, box_k, 128) &&
             map_2d(&m.w3, w->w3, fp8, H, (uint64_t)E * I, box_k, 128) &&
             map_2d(&m.h, ws + L.h, fp8, I, R, box_k, kTileM) &&
-            map_2d(&m.w2, w->w2, fp8, I, (uint64_t)E * H, box_k, 128);
+            map_2d(&m.w2, w->w2, fp8, I, (uint64_t)E * H, box_k, 256) &&
+            map_2d(&m.w2h, w->w2, fp8, I, (uint64_t)E * H, box_k, 128);
   if (S) {
     ok = ok && map_2d(&m.sw1, w->sw1, fp8, H, I, box_k, 128) && map_2d(&m.sw3, w->sw3, fp8, H, I, box_k, 128) &&
-         map_2d(&m.sw2, w->sw2, fp8, I, H, box_k, 128);
+         map_2d(&m.sw2, w->sw2, fp8, I, H, box_k, 256) && map_2d(&m.sw2h, w->sw2, fp8, I, H, box_k, 128);
   } else {
     m.sw1 = m.w1;
     m.sw3 = m.w3;
     m.sw2 = m.w2;
+    m.sw2h = m.w2h;
   }
   if (!ok) return MOE_ERR_CUDA;
 
@@ -289,7 +291,7 @@ int run_experts(const moe_config* c, const WsLayout& L, int64_t T, const void* x
   g2.out = y;
   g2.out_scale = nullptr;
   g2.row_gate = reinterpret_cast<const float*>(ws + L.row_gate);
-  CUDA_TRY(launch_gemm2(g2, fp8, pair, sms, m.h, m.w2, m.sw2, s));
+  CUDA_TRY(launch_gemm2(g2, fp8, pair, sms, m.h, m.w2, m.w2h, m.sw2, m.sw2h, s));
   prof.mark();
   return MOE_OK;
 }

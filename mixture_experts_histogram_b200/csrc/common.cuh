@@ -118,8 +118,10 @@ cudaError_t launch_gather(const GatherParams& p, bool fp8, cudaStream_t s);
 cudaError_t launch_gemm1(const GemmParams& p, bool fp8, bool pair, int grid, const CUtensorMap& tm_a,
                          const CUtensorMap& tm_w1, const CUtensorMap& tm_w3, const CUtensorMap& tm_sw1,
                          const CUtensorMap& tm_sw3, cudaStream_t s);
+// tm_w2 / tm_sw2 use 256-row boxes, tm_w2h / tm_sw2h the same tensors with 128-row boxes.
 cudaError_t launch_gemm2(const GemmParams& p, bool fp8, bool pair, int grid, const CUtensorMap& tm_a,
-                         const CUtensorMap& tm_w2, const CUtensorMap& tm_sw2, cudaStream_t s);
+                         const CUtensorMap& tm_w2, const CUtensorMap& tm_w2h, const CUtensorMap& tm_sw2,
+                         const CUtensorMap& tm_sw2h, cudaStream_t s);
 cudaError_t launch_combine(const CombineParams& p, cudaStream_t s);
 
 }  // namespace moe

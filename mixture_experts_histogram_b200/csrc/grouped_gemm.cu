@@ -113,7 +113,9 @@ __device__ __forceinline__ Item decode_item(int item, int n_tiles, int G, int ti
 }
 
 // Weight-tile rows of a work item: box 0 starts at row `yb` of `*m0`, box 1 at
-// row `yb2` of `*m1` (GEMM1: W1 and W3 rows n0..; GEMM2: W2 rows n0.. and n0+128..).
+// row `yb2` of `*m1`. GEMM1: W1 and W3 rows n0.. (128-row boxes). GEMM2: `*m0`
+// maps W2 with 256-row boxes (rows n0..n0+255 in one load), `*m1` the same W2
+// with 128-row boxes (the 2-SM variant loads rows n0.. and n0+128.. per CTA).
 template <bool kGemm1>
 struct BRows {
   const CUtensorMap *m0, *m1;
@@ -123,7 +125,7 @@ struct BRows {
     const bool shared = (it.g == p.E);
     yb = (shared ? 0 : it.g * p.N) + it.n * (kGemm1 ? 128 : 256);
     m0 = shared ? bs0 : b0;
-    m1 = kGemm1 ? (shared ? bs1 : b1) : m0;
+    m1 = shared ? bs1 : b1;  // GEMM1: W3; GEMM2: the same W2 with 128-row boxes
     yb2 = kGemm1 ? yb : yb + 128;
   }
 };
@@ -202,10 +204,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     tma_prefetch_desc(&tm_a);
     tma_prefetch_desc(&tm_b0);
     tma_prefetch_desc(&tm_bs0);
-    if (kGemm1) {
-      tma_prefetch_desc(&tm_b1);
-      tma_prefetch_desc(&tm_bs1);
-    }
+    tma_prefetch_desc(&tm_b1);
+    tma_prefetch_desc(&tm_bs1);
   }
   if (warp == 1) {
     if (kPair) {
@@ -273,12 +273,19 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t bar0 = map_to_cta(&full[stage], 0);
             if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2 * C::kStageBytes);
             tma_load_2d_pair(sA + stage * kABytes, &tm_a, bar0, kx, my_row0);
-            tma_load_2d_pair(sB + stage * C::kBBytes, rank ? rows.m1 : rows.m0, bar0, kx, rank ? rows.yb2 : rows.yb);
+            // GEMM2's 128-row halves come from the 128-row-box map (passed as the second map).
+            tma_load_2d_pair(sB + stage * C::kBBytes, (kGemm1 && rank == 0) ? rows.m0 : rows.m1, bar0, kx,
+                             rank ? rows.yb2 : rows.yb);
           } else {
             mbar_arrive_expect_tx(&full[stage], C::kStageBytes);
             tma_load_2d(sA + stage * kABytes, &tm_a, &full[stage], kx, my_row0);
-            tma_load_2d(sB + stage * C::kBBytes, rows.m0, &full[stage], kx, rows.yb);
-            tma_load_2d(sB + stage * C::kBBytes + C::kBBytes / 2, rows.m1, &full[stage], kx, rows.yb2);
+            if (kGemm1) {
+              tma_load_2d(sB + stage * C::kBBytes, rows.m0, &full[stage], kx, rows.yb);
+              tma_load_2d(sB + stage * C::kBBytes + C::kBBytes / 2, rows.m1, &full[stage], kx, rows.yb2);
+            } else {
+              // GEMM2's 256 weight rows are contiguous: one 256-row box.
+              tma_load_2d(sB + stage * C::kBBytes, rows.m0, &full[stage], kx, rows.yb);
+            }
           }
           issued |= 1u << stage;
           issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
@@ -599,12 +606,13 @@ cudaError_t launch_gemm1(const GemmParams& p, bool fp8, bool pair, int grid, con
 }
 
 cudaError_t launch_gemm2(const GemmParams& p, bool fp8, bool pair, int grid, const CUtensorMap& tm_a,
-                         const CUtensorMap& tm_w2, const CUtensorMap& tm_sw2, cudaStream_t s) {
+                         const CUtensorMap& tm_w2, const CUtensorMap& tm_w2h, const CUtensorMap& tm_sw2,
+                         const CUtensorMap& tm_sw2h, cudaStream_t s) {
   if (pair)
-    return fp8 ? launch_one<true, false, true>(p, grid, tm_a, tm_w2, tm_w2, tm_sw2, tm_sw2, s)
-               : launch_one<false, false, true>(p, grid, tm_a, tm_w2, tm_w2, tm_sw2, tm_sw2, s);
-  return fp8 ? launch_one<true, false, false>(p, grid, tm_a, tm_w2, tm_w2, tm_sw2, tm_sw2, s)
-             : launch_one<false, false, false>(p, grid, tm_a, tm_w2, tm_w2, tm_sw2, tm_sw2, s);
+    return fp8 ? launch_one<true, false, true>(p, grid, tm_a, tm_w2, tm_w2h, tm_sw2, tm_sw2h, s)
+               : launch_one<false, false, true>(p, grid, tm_a, tm_w2, tm_w2h, tm_sw2, tm_sw2h, s);
+  return fp8 ? launch_one<true, false, false>(p, grid, tm_a, tm_w2, tm_w2h, tm_sw2, tm_sw2h, s)
+             : launch_one<false, false, false>(p, grid, tm_a, tm_w2, tm_w2h, tm_sw2, tm_sw2h, s);
 }
 
 }  // namespace moe
