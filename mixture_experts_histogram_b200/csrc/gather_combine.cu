@@ -36,34 +36,54 @@ __global__ void __launch_bounds__(256) gather_bf16_kernel(const GatherParams p) 
   }
 }
 
-// One warp per 128-element block; each lane quantises 4 consecutive values.
+// One half-warp per 128-element block: each lane loads 8 bf16 (16 bytes),
+// the half-warp reduces the block's amax, and each lane stores its 8 codes
+// (8 bytes) to every destination row.
+template <int kMaxSlots>
 __global__ void __launch_bounds__(256) gather_fp8_kernel(const GatherParams p) {
   const int64_t t = blockIdx.x;
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int half = lane / 16, hl = lane % 16;
   const int nblk = p.H / 128;
-  for (int kb = warp; kb < nblk; kb += 8) {
-    const uint2 raw = *reinterpret_cast<const uint2*>(p.x + t * p.H + kb * 128 + lane * 4);
-    const __nv_bfloat162 b01 = *reinterpret_cast<const __nv_bfloat162*>(&raw.x);
-    const __nv_bfloat162 b23 = *reinterpret_cast<const __nv_bfloat162*>(&raw.y);
-    const float2 f01 = __bfloat1622float2(b01), f23 = __bfloat1622float2(b23);
-    float amax = fmaxf(fmaxf(fabsf(f01.x), fabsf(f01.y)), fmaxf(fabsf(f23.x), fabsf(f23.y)));
+  int32_t rows[kMaxSlots];  // destination rows (< 2^31)
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+  for (int j = 0; j < kMaxSlots; ++j) rows[j] = j < p.S ? (p.pos ? p.pos[t * p.S + j] : (int32_t)t) : -1;
+  for (int kb0 = 2 * warp; kb0 < nblk; kb0 += 16) {
+    const int kb = kb0 + half;
+    const bool active = kb < nblk;
+    uint4 raw = make_uint4(0, 0, 0, 0);
+    if (active) raw = __ldcs(reinterpret_cast<const uint4*>(p.x + t * p.H + kb * 128) + hl);
+    const __nv_bfloat162* b = reinterpret_cast<const __nv_bfloat162*>(&raw);
+    float f[8];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float2 v = __bfloat1622float2(b[i]);
+      f[2 * i] = v.x;
+      f[2 * i + 1] = v.y;
+    }
+    float amax = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(f[i]));
+#pragma unroll
+    for (int off = 8; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
     float s = 1.0f;
-    uint32_t codes = 0;
+    uint2 codes = make_uint2(0, 0);
     if (amax > 0.0f) {
       s = __fdiv_rn(amax, 448.0f);
-      const float2 q01 = make_float2(__fdiv_rn(f01.x, s), __fdiv_rn(f01.y, s));
-      const float2 q23 = make_float2(__fdiv_rn(f23.x, s), __fdiv_rn(f23.y, s));
-      const uint32_t lo = __nv_cvt_float2_to_fp8x2(q01, __NV_SATFINITE, __NV_E4M3);
-      const uint32_t hi = __nv_cvt_float2_to_fp8x2(q23, __NV_SATFINITE, __NV_E4M3);
-      codes = lo | (hi << 16);
+      uint32_t w[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        w[i] = __nv_cvt_float2_to_fp8x2(make_float2(__fdiv_rn(f[2 * i], s), __fdiv_rn(f[2 * i + 1], s)),
+                                        __NV_SATFINITE, __NV_E4M3);
+      codes = make_uint2(w[0] | (w[1] << 16), w[2] | (w[3] << 16));
     }
-    for (int j = 0; j < p.S; ++j) {
-      const int64_t row = p.pos ? p.pos[t * p.S + j] : t;
+    if (!active) continue;
+#pragma unroll
+    for (int j = 0; j < kMaxSlots; ++j) {
+      const int64_t row = rows[j];
       if (row < 0) continue;
-      *reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(p.xp) + row * p.H + kb * 128 + lane * 4) = codes;
-      if (lane == 0) {
+      *reinterpret_cast<uint2*>(static_cast<uint8_t*>(p.xp) + row * p.H + kb * 128 + hl * 8) = codes;
+      if (hl == 0) {
         if (p.scale_row_major) p.sxp[row * nblk + kb] = s;
         else p.sxp[(int64_t)kb * p.rows_pad + row] = s;
       }
@@ -71,18 +91,28 @@ __global__ void __launch_bounds__(256) gather_fp8_kernel(const GatherParams p) {
   }
 }
 
+// One CTA per token. Each thread owns 8 output columns per step; the token's
+// row indices live in registers and every row's 16-byte chunk is loaded before
+// the sum, so up to kMaxSlots independent loads are in flight per thread.
+template <int kMaxSlots>
 __global__ void __launch_bounds__(256) combine_kernel(const CombineParams p) {
   const int64_t t = blockIdx.x;
   const int nvec = p.H / 8;
+  int32_t rows[kMaxSlots];
+#pragma unroll
+  for (int j = 0; j < kMaxSlots; ++j) rows[j] = j < p.S ? p.pos[t * p.S + j] : -1;
   for (int c = threadIdx.x; c < nvec; c += blockDim.x) {
+    uint4 v[kMaxSlots];
+#pragma unroll
+    for (int j = 0; j < kMaxSlots; ++j)
+      if (rows[j] >= 0) v[j] = __ldcs(reinterpret_cast<const uint4*>(p.y + (int64_t)rows[j] * p.H) + c);
     float acc[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) acc[i] = 0.0f;
-    for (int j = 0; j < p.S; ++j) {
-      const int64_t r = p.pos[t * p.S + j];
-      if (r < 0) continue;
-      const uint4 v = reinterpret_cast<const uint4*>(p.y + r * p.H)[c];
-      const __nv_bfloat162* b = reinterpret_cast<const __nv_bfloat162*>(&v);
+#pragma unroll
+    for (int j = 0; j < kMaxSlots; ++j) {  // slot order: routed slots, then the shared expert
+      if (rows[j] < 0) continue;
+      const __nv_bfloat162* b = reinterpret_cast<const __nv_bfloat162*>(&v[j]);
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         const float2 f = __bfloat1622float2(b[i]);
@@ -102,14 +132,16 @@ __global__ void __launch_bounds__(256) combine_kernel(const CombineParams p) {
 
 cudaError_t launch_gather(const GatherParams& p, bool fp8, cudaStream_t s) {
   if (p.T == 0) return cudaSuccess;
-  if (fp8) gather_fp8_kernel<<<(unsigned)p.T, 256, 0, s>>>(p);
+  if (fp8 && p.S <= 9) gather_fp8_kernel<9><<<(unsigned)p.T, 256, 0, s>>>(p);
+  else if (fp8) gather_fp8_kernel<kMaxTopK + 1><<<(unsigned)p.T, 256, 0, s>>>(p);
   else gather_bf16_kernel<<<(unsigned)p.T, 256, 0, s>>>(p);
   return cudaGetLastError();
 }
 
 cudaError_t launch_combine(const CombineParams& p, cudaStream_t s) {
   if (p.T == 0) return cudaSuccess;
-  combine_kernel<<<(unsigned)p.T, 256, 0, s>>>(p);
+  if (p.S <= 9) combine_kernel<9><<<(unsigned)p.T, 256, 0, s>>>(p);
+  else combine_kernel<kMaxTopK + 1><<<(unsigned)p.T, 256, 0, s>>>(p);
   return cudaGetLastError();
 }
 
