@@ -9,7 +9,8 @@
 // tiles with TMA into a 3-4 stage ring of 128B-swizzled shared-memory tiles;
 // warp 1 issues tcgen05 MMAs (M = 128 tokens, N = up to 2 x 256 experts) into a
 // TMEM accumulator; warps 2-5 read the accumulator back (one token row per
-// thread) and store fp32 partial logits. Small T is split along K so that the
+// thread, 32 columns at a time), transpose each 32 x 32 block through shared
+// memory and store fp32 partial logits as whole 128-byte row segments. Small T is split along K so that the
 // 2.9 MB of router weights are streamed by many SMs at once; the top-k kernel
 // adds the K-split partials in a fixed order.
 #include <cuda_bf16.h>
@@ -118,21 +119,26 @@ __global__ void __launch_bounds__(kRouterThreads, 1)
   } else if (warp >= 2) {
     // ---- epilogue: one token row per thread ----
     const int q = warp % 4;
-    const int row = m_tile * kTileM + q * 32 + lane;
     bool ok = mbar_wait(done, 0, p.status, abort_flag);
     ok = __all_sync(0xffffffffu, ok);
     if (ok) {
       tc_fence_after_sync();
-      float* dst = p.partial + ((int64_t)split * p.T + row) * p.E;
+      // Every MMA has completed (done), so the stage buffers are free: each
+      // warp transposes through its own 32 x 33 float block of them.
+      float* tr = reinterpret_cast<float*>(smem) + (warp - 2) * 32 * 33;
+      const int row0 = m_tile * kTileM + q * 32;  // first token row of this warp
+      float* dst0 = p.partial + ((int64_t)split * p.T + row0) * p.E;
       for (int c0 = 0; c0 < ncols; c0 += 32) {
         uint32_t v[32];
         tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)c0, v);
         tmem_ld_wait();
-        if (row < p.T) {
 #pragma unroll
-          for (int i = 0; i < 32; ++i)
-            if (c0 + i < p.E) dst[c0 + i] = __uint_as_float(v[i]);
-        }
+        for (int i = 0; i < 32; ++i) tr[lane * 33 + i] = __uint_as_float(v[i]);
+        __syncwarp();
+        const int c = c0 + lane;
+        for (int r = 0; r < 32 && row0 + r < p.T; ++r)
+          if (c < p.E) dst0[(int64_t)r * p.E + c] = tr[r * 33 + lane];
+        __syncwarp();
       }
     }
   }
@@ -153,17 +159,34 @@ __global__ void __launch_bounds__(256) topk_kernel(const TopkParams p) {
   if (t >= p.T) return;
   constexpr int kPer = kMaxExperts / 32;
   float l[kPer];
+  // The loads of up to four splits are independent and issued together; the
+  // splits are added in split order.
+  const float* __restrict__ part = p.partial;
+#pragma unroll
+  for (int i = 0; i < kPer; ++i) l[i] = (lane + 32 * i < p.E) ? 0.0f : -INFINITY;
+  constexpr int kSplitBatch = 4;
+  for (int s0 = 0; s0 < p.ksplit; s0 += kSplitBatch) {
+    float v[kSplitBatch][kPer];
+#pragma unroll
+    for (int u = 0; u < kSplitBatch; ++u) {
+      const float* src = part + ((int64_t)(s0 + u) * p.T + t) * p.E;
+#pragma unroll
+      for (int i = 0; i < kPer; ++i)
+        v[u][i] = (s0 + u < p.ksplit && lane + 32 * i < p.E) ? __ldg(src + lane + 32 * i) : 0.0f;
+    }
+#pragma unroll
+    for (int u = 0; u < kSplitBatch; ++u)
+#pragma unroll
+      for (int i = 0; i < kPer; ++i)
+        if (s0 + u < p.ksplit) l[i] += v[u][i];
+  }
 #pragma unroll
   for (int i = 0; i < kPer; ++i) {
     const int e = lane + 32 * i;
-    float v = -INFINITY;
     if (e < p.E) {
-      v = 0.0f;
-      for (int s = 0; s < p.ksplit; ++s) v += p.partial[((int64_t)s * p.T + t) * p.E + e];
-      if (p.bias) v += p.bias[e];
-      if (p.logits) p.logits[t * p.E + e] = v;
+      if (p.bias) l[i] += __ldg(p.bias + e);
+      if (p.logits) p.logits[t * p.E + e] = l[i];
     }
-    l[i] = v;
   }
   uint32_t taken = 0;
   float my_v = -INFINITY;
