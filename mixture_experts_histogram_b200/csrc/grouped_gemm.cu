@@ -130,7 +130,11 @@ struct BRows {
   }
 };
 
-__device__ __forceinline__ float silu_mul(float g, float u) { return g / (1.0f + __expf(-g)) * u; }
+// silu(g) * u. The quotient uses the fast division: exact IEEE division falls
+// into its slow path whenever exp(-g) overflows (rows of a tile past its
+// group's end can hold large values), which once cost a fifth of GEMM1's time.
+// For an infinite denominator the fast quotient is 0, silu's limit.
+__device__ __forceinline__ float silu_mul(float g, float u) { return __fdividef(g, 1.0f + __expf(-g)) * u; }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
   const __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
