@@ -214,8 +214,10 @@ MOE_API const char* moe_profile_kernel_name(int i);
 
 /* Expert-GEMM variant (process-wide; default MOE_GEMM_AUTO). SINGLE runs one
  * CTA per 128-row tile; PAIR runs 2-SM CTA pairs on 256-row tiles (each weight
- * tile crosses L2 -> SM once per 256 rows). AUTO currently runs SINGLE, the
- * faster of the two for FP8 experts. All variants compute the same result. */
+ * tile crosses L2 -> SM once per 256 rows). AUTO runs the gate/up GEMM on pairs
+ * when top_k * T >= 128 * n_experts (routed groups of 128+ rows on average) and
+ * everything else on single CTAs. All variants compute the same layer and are
+ * held to the same tolerance by the tests. */
 enum { MOE_GEMM_AUTO = 0, MOE_GEMM_SINGLE = 1, MOE_GEMM_PAIR = 2 };
 MOE_API int moe_set_gemm_variant(int variant);
 

@@ -16,11 +16,14 @@ namespace {
 // CTAs the router aims for when it splits K for small token counts (B200: 148 SMs).
 constexpr int kRouterTargetCtas = 148;
 
-// Expert-GEMM variant. AUTO runs the single-CTA kernels: with FP8 experts the
-// 2-SM pair needs a TMEM hand-off between the MMA and both SMs' epilogues for
-// every 128-deep K block, and that cross-SM round trip made it slower than
-// the single-CTA kernel at T = 8192 (2.72 vs 1.56 ms for the gate/up GEMM).
+// Expert-GEMM variant. AUTO runs GEMM1 (gate/up) on 2-SM pairs when the
+// routed groups average at least kPairMinRows rows (prefill: each weight tile
+// then crosses L2 -> SM once per 256 rows; 1.46 vs 1.57 ms at T = 8192) and
+// on single CTAs otherwise (decode: a 256-row tile would load twice the
+// activation rows for one or two valid ones). GEMM2 (down) runs on single CTAs,
+// which measured faster at every size (0.91 vs 0.98 ms at T = 8192).
 int g_gemm_variant = MOE_GEMM_AUTO;
+constexpr int64_t kPairMinRows = 128;
 
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 std::once_flag g_encode_once;
@@ -222,7 +225,8 @@ int run_experts(const moe_config* c, const WsLayout& L, int64_t T, const void* x
   const int64_t R = L.R;
   const int sms = sm_count();
   if (sms <= 0) return MOE_ERR_CUDA;
-  const bool pair = g_gemm_variant == MOE_GEMM_PAIR;
+  const bool pair = g_gemm_variant == MOE_GEMM_PAIR;  // GEMM2 (and the maps it shares)
+  const bool pair1 = pair || (g_gemm_variant == MOE_GEMM_AUTO && (int64_t)c->top_k * T >= kPairMinRows * E);
 
   GatherParams gp{};
   gp.T = (int32_t)T;
@@ -256,7 +260,7 @@ int run_experts(const moe_config* c, const WsLayout& L, int64_t T, const void* x
   if (!ok) return MOE_ERR_CUDA;
 
   GemmParams g1{};
-  g1.mt_prefix = reinterpret_cast<const int32_t*>(ws + (pair ? L.mp_prefix : L.mt_prefix));
+  g1.mt_prefix = reinterpret_cast<const int32_t*>(ws + (pair1 ? L.mp_prefix : L.mt_prefix));
   g1.offsets = reinterpret_cast<const int32_t*>(ws + L.offsets);
   g1.G = E + S;
   g1.E = E;
@@ -275,10 +279,11 @@ int run_experts(const moe_config* c, const WsLayout& L, int64_t T, const void* x
   g1.out_scale = fp8 ? reinterpret_cast<float*>(ws + L.sh) : nullptr;
   g1.row_gate = nullptr;
   g1.status = reinterpret_cast<int*>(ws + L.status);
-  CUDA_TRY(launch_gemm1(g1, fp8, pair, sms, m.xp, m.w1, m.w3, m.sw1, m.sw3, s));
+  CUDA_TRY(launch_gemm1(g1, fp8, pair1, sms, m.xp, m.w1, m.w3, m.sw1, m.sw3, s));
   prof.mark();
 
   GemmParams g2 = g1;
+  g2.mt_prefix = reinterpret_cast<const int32_t*>(ws + (pair ? L.mp_prefix : L.mt_prefix));
   g2.K = I;
   g2.N = H;
   g2.n_tiles = (int32_t)ceil_div(H, 256);

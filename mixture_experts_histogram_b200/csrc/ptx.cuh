@@ -170,8 +170,12 @@ __device__ __forceinline__ uint32_t map_to_cta(const void* p, uint32_t cta) {
 }
 
 // Arrive on an mbarrier given by its shared::cluster address (possibly a peer's).
+// Release at CTA scope only: the arrivals this is used for (TMEM partial freed)
+// follow a tcgen05.wait::ld, so there is no memory write to publish, and a
+// cluster-scope release (a cluster-wide fence per arrival) measured at half of
+// the 2-SM epilogue's time.
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+  asm volatile("mbarrier.arrive.release.cta.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
 
 __device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t parity) {

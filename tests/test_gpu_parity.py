@@ -293,6 +293,12 @@ def _layer_cases():
                         wdtype=synth.WDTYPE_FP8, seed=16), None),
         (synth.MoeShape("E512-k16-fp8", T=160, hidden=256, n_experts=512, top_k=16, n_shared=1, inter=128,
                         wdtype=synth.WDTYPE_FP8, seed=17), None),
+        # top_k * T >= 128 * E: the automatic choice runs the gate/up GEMM on 2-SM
+        # pairs and the down GEMM on single CTAs.
+        (synth.MoeShape("auto-pair-fp8", T=600, hidden=512, n_experts=8, top_k=2, n_shared=1, inter=256,
+                        wdtype=synth.WDTYPE_FP8, seed=24), None),
+        (synth.MoeShape("auto-pair-bf16", T=520, hidden=384, n_experts=6, top_k=2, n_shared=0, inter=384,
+                        seed=25), None),
         (synth.DECODE_BF16, None),
         (synth.SWEEP_FP8.with_tokens(1), None),
         (synth.SWEEP_FP8.with_tokens(8), None),
