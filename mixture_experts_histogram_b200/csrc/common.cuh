@@ -109,6 +109,7 @@ struct CombineParams {
 cudaError_t launch_router_gemm(const RouterParams& p, const CUtensorMap& tm_x, const CUtensorMap& tm_w,
                                cudaStream_t s);
 cudaError_t launch_topk(const TopkParams& p, cudaStream_t s);
+cudaError_t launch_permute_one_chunk(const PermuteParams& p, cudaStream_t s);  // T <= 256
 cudaError_t launch_histogram(const PermuteParams& p, cudaStream_t s);
 cudaError_t launch_scan(const PermuteParams& p, cudaStream_t s);
 cudaError_t launch_scatter(const PermuteParams& p, cudaStream_t s);

@@ -18,6 +18,8 @@
 //      warps are then offset by an exclusive scan over the CTA's 8 warps, and
 //      rows are written: perm[row] = token, pos[token, slot] = row,
 //      row_gate[row] = gate.
+// With a single chunk (T <= 256, decode) one CTA runs the three steps in one
+// launch, with block barriers between them.
 #include "common.cuh"
 #include "ptx.cuh"
 
@@ -25,11 +27,10 @@ namespace moe {
 
 namespace {
 
-__global__ void __launch_bounds__(256) histogram_kernel(const PermuteParams p) {
-  __shared__ int cnt[kMaxExperts];
+__device__ __forceinline__ void histogram_block(const PermuteParams& p, int chunk, int* cnt) {
   for (int e = threadIdx.x; e < p.E; e += blockDim.x) cnt[e] = 0;
   __syncthreads();
-  const int64_t t0 = (int64_t)blockIdx.x * kHistChunk;
+  const int64_t t0 = (int64_t)chunk * kHistChunk;
   const int64_t ntok = min((int64_t)kHistChunk, (int64_t)p.T - t0);
   const int64_t npairs = ntok * p.k;
   const int32_t* idx = p.idx + t0 * p.k;
@@ -39,7 +40,12 @@ __global__ void __launch_bounds__(256) histogram_kernel(const PermuteParams p) {
     else atomicAdd(&cnt[e], 1);
   }
   __syncthreads();
-  for (int e = threadIdx.x; e < p.E; e += blockDim.x) p.chunk_base[(int64_t)e * p.chunks + blockIdx.x] = cnt[e];
+  for (int e = threadIdx.x; e < p.E; e += blockDim.x) p.chunk_base[(int64_t)e * p.chunks + chunk] = cnt[e];
+}
+
+__global__ void __launch_bounds__(256) histogram_kernel(const PermuteParams p) {
+  __shared__ int cnt[kMaxExperts];
+  histogram_block(p, blockIdx.x, cnt);
 }
 
 __device__ __forceinline__ int warp_inclusive_scan(int v, int lane) {
@@ -51,12 +57,10 @@ __device__ __forceinline__ int warp_inclusive_scan(int v, int lane) {
   return v;
 }
 
-__global__ void __launch_bounds__(1024) scan_kernel(const PermuteParams p) {
-  __shared__ int cnt_s[kMaxExperts + 1];
-  __shared__ int off_s[kMaxExperts + 2];
-  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+__device__ __forceinline__ void scan_block(const PermuteParams& p, int* cnt_s, int* off_s) {
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32, nwarps = blockDim.x / 32;
   // per-expert exclusive scan over chunks (bases relative to the expert)
-  for (int e = warp; e < p.E; e += 32) {
+  for (int e = warp; e < p.E; e += nwarps) {
     int running = 0;
     int32_t* row = p.chunk_base + (int64_t)e * p.chunks;
     for (int c0 = 0; c0 < p.chunks; c0 += 32) {
@@ -103,13 +107,18 @@ __global__ void __launch_bounds__(1024) scan_kernel(const PermuteParams p) {
   for (int64_t i = threadIdx.x; i < n; i += blockDim.x) p.chunk_base[i] += off_s[i / p.chunks];
 }
 
-__global__ void __launch_bounds__(256) scatter_kernel(const PermuteParams p) {
-  __shared__ int wcnt[8][kMaxExperts];
+__global__ void __launch_bounds__(1024) scan_kernel(const PermuteParams p) {
+  __shared__ int cnt_s[kMaxExperts + 1];
+  __shared__ int off_s[kMaxExperts + 2];
+  scan_block(p, cnt_s, off_s);
+}
+
+__device__ __forceinline__ void scatter_block(const PermuteParams& p, int chunk, int (*wcnt)[kMaxExperts]) {
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   for (int i = threadIdx.x; i < 8 * kMaxExperts; i += blockDim.x) (&wcnt[0][0])[i] = 0;
   __syncthreads();
 
-  const int64_t tw0 = (int64_t)blockIdx.x * kHistChunk + warp * 32;  // this warp's first token
+  const int64_t tw0 = (int64_t)chunk * kHistChunk + warp * 32;  // this warp's first token
   int rank[kMaxTopK];
   int ekeep[kMaxTopK];
   // Pass 1: ranks inside the warp, pairs taken in (token, slot) order, 32 per round.
@@ -140,7 +149,7 @@ __global__ void __launch_bounds__(256) scatter_kernel(const PermuteParams p) {
   __syncthreads();
   // Pass 2: warp offsets per expert, on top of this chunk's absolute base.
   for (int e = threadIdx.x; e < p.E; e += blockDim.x) {
-    int run = p.chunk_base[(int64_t)e * p.chunks + blockIdx.x];
+    int run = p.chunk_base[(int64_t)e * p.chunks + chunk];
 #pragma unroll
     for (int w = 0; w < 8; ++w) {
       const int v = wcnt[w][e];
@@ -172,7 +181,7 @@ __global__ void __launch_bounds__(256) scatter_kernel(const PermuteParams p) {
   }
   // The shared expert's rows: token order.
   if (p.S) {
-    const int64_t t = (int64_t)blockIdx.x * kHistChunk + threadIdx.x;
+    const int64_t t = (int64_t)chunk * kHistChunk + threadIdx.x;
     if (t < p.T) {
       const int row = p.offsets[p.E] + (int)t;
       p.perm[row] = (int32_t)t;
@@ -182,7 +191,65 @@ __global__ void __launch_bounds__(256) scatter_kernel(const PermuteParams p) {
   }
 }
 
+__global__ void __launch_bounds__(256) scatter_kernel(const PermuteParams p) {
+  __shared__ int wcnt[8][kMaxExperts];
+  scatter_block(p, blockIdx.x, wcnt);
+}
+
+// T <= 256: the three steps in one CTA. With a single chunk the per-expert
+// chunk scan is the identity, so the counts come straight from the shared
+// histogram, one warp scans them over the groups, and the scatter follows. The
+// block barriers also make each step's global writes visible to the next.
+__global__ void __launch_bounds__(256) permute_one_chunk_kernel(const PermuteParams p) {
+  __shared__ int wcnt[8][kMaxExperts];  // scatter; rows 0-1 first hold the expert counts
+  int* cnt = &wcnt[0][0];
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  for (int e = threadIdx.x; e < p.E; e += blockDim.x) cnt[e] = 0;
+  __syncthreads();
+  const int npairs = p.T * p.k;
+  for (int i = threadIdx.x; i < npairs; i += blockDim.x) {
+    const int e = p.idx[i];
+    if (e < 0 || e >= p.E) latch_status(p.status, MOE_ERR_BAD_INDEX);
+    else atomicAdd(&cnt[e], 1);
+  }
+  __syncthreads();
+  if (warp == 0) {
+    int run_off = 0, run_mt = 0, run_mp = 0;
+    for (int g0 = 0; g0 < p.G; g0 += 32) {
+      const int g = g0 + lane;
+      const int c = g < p.E ? cnt[g] : (g < p.G ? p.T : 0);  // group E: the shared expert
+      const int mt = (c + kTileM - 1) / kTileM;
+      const int mp = (c + 2 * kTileM - 1) / (2 * kTileM);
+      const int ic = warp_inclusive_scan(c, lane);
+      const int im = warp_inclusive_scan(mt, lane);
+      const int ip = warp_inclusive_scan(mp, lane);
+      if (g < p.G) {
+        p.counts[g] = c;
+        p.offsets[g] = run_off + ic - c;
+        p.mt_prefix[g] = run_mt + im - mt;
+        p.mp_prefix[g] = run_mp + ip - mp;
+        if (g < p.E) p.chunk_base[g] = run_off + ic - c;  // the one chunk starts at the group's offset
+      }
+      run_off += __shfl_sync(0xffffffffu, ic, 31);
+      run_mt += __shfl_sync(0xffffffffu, im, 31);
+      run_mp += __shfl_sync(0xffffffffu, ip, 31);
+    }
+    if (lane == 0) {
+      p.offsets[p.G] = run_off;
+      p.mt_prefix[p.G] = run_mt;
+      p.mp_prefix[p.G] = run_mp;
+    }
+  }
+  __syncthreads();
+  scatter_block(p, 0, wcnt);
+}
+
 }  // namespace
+
+cudaError_t launch_permute_one_chunk(const PermuteParams& p, cudaStream_t s) {
+  permute_one_chunk_kernel<<<1, 256, 0, s>>>(p);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_histogram(const PermuteParams& p, cudaStream_t s) {
   histogram_kernel<<<p.chunks, 256, 0, s>>>(p);
