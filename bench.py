@@ -223,21 +223,30 @@ def run_ours(args):
         if world > 1:
             dist.barrier()
         torch.cuda.synchronize()
-        m.moe_profile_enable(profile)
+        # Timed steps: no per-kernel events inside. Before each step ~1 ms of GPU
+        # sleep (outside ev0..ev1) lets the host queue the whole step, so the
+        # device time is not stretched by host launch gaps.
         for i in range(args.steps):
             flush.fill_(i & 0xFF)
-            torch.cuda._sleep(200000)  # ~0.1 ms of GPU time so the host has queued the step before ev0
+            torch.cuda._sleep(2000000)
             ev[i][0].record(stream)
             step()
             ev[i][1].record(stream)
-            if profile:
-                for k, v in m.moe_profile_read().items():
-                    per_kernel[k] += v
         torch.cuda.synchronize()
-        m.moe_profile_enable(False)
         if world > 1:
             dist.barrier()
         total_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in ev), world, f"cuda:{local}")
+        if profile:
+            # Per-kernel split from a separate pass with an event between kernels.
+            m.moe_profile_enable(True)
+            for i in range(args.steps):
+                flush.fill_(i & 0xFF)
+                torch.cuda._sleep(2000000)
+                step()
+                for k, v in m.moe_profile_read().items():
+                    per_kernel[k] += v
+            torch.cuda.synchronize()
+            m.moe_profile_enable(False)
         st = m.moe_read_status(ws)
         if st != 0:
             raise RuntimeError(f"device status after timing: {m.moe_status_string(st)}")
