@@ -481,21 +481,44 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_fence_after_sync();
           const uint32_t base = tmem + lane_base + b * 256;
           constexpr int kNch = 128 / kFp8Chunk;  // chunks per thread per K block
-#pragma unroll
-          for (int ch = 0; ch < kNch; ++ch) {
-            uint32_t v[kFp8Chunk];
-            const int c = ch * kFp8Chunk;  // 0..127 within this thread's 128 columns
-            const uint32_t col = kGemm1 ? (c < 64 ? 0u : 128u) + 64 * hf + (c & 63) : 128 * hf + c;
-            if constexpr (kFp8Chunk == 32) tmem_ld32(base + col, v);
-            else tmem_ld16(base + col, v);
-            tmem_ld_wait();
-            if (ch == kNch - 1) release_acc(b);
+          auto col_of = [&](int ch) -> uint32_t {
+            const int c = ch * kFp8Chunk;
+            return kGemm1 ? (c < 64 ? 0u : 128u) + 64 * hf + (c & 63) : 128 * hf + c;
+          };
+          auto promote = [&](const uint32_t (&v)[kFp8Chunk], int ch) {
+            const int c = ch * kFp8Chunk;
             const float f = (kGemm1 && c >= 64) ? f1 : f0;
             const float2 ff = make_float2(f, f);
 #pragma unroll
             for (int i = 0; i < kFp8Chunk / 2; ++i)
               acc[c / 2 + i] = fma2(make_float2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1])), ff,
                                     acc[c / 2 + i]);
+          };
+          if constexpr (kGemm1) {
+            // Two load buffers: the next chunk's load is in flight while the
+            // current one is promoted (GEMM1: 1.5% faster; GEMM2 measured slower).
+            uint32_t va[kFp8Chunk], vb[kFp8Chunk];
+            tmem_ld16(base + col_of(0), va);
+            tmem_ld_wait(va);
+#pragma unroll
+            for (int ch = 0; ch < kNch; ch += 2) {
+              tmem_ld16(base + col_of(ch + 1), vb);
+              promote(va, ch);
+              tmem_ld_wait(vb);
+              if (ch + 2 < kNch) tmem_ld16(base + col_of(ch + 2), va);
+              else release_acc(b);  // every load of this partial has completed
+              promote(vb, ch + 1);
+              if (ch + 2 < kNch) tmem_ld_wait(va);
+            }
+          } else {
+#pragma unroll
+            for (int ch = 0; ch < kNch; ++ch) {
+              uint32_t v[kFp8Chunk];
+              tmem_ld16(base + col_of(ch), v);
+              tmem_ld_wait(v);
+              if (ch == kNch - 1) release_acc(b);
+              promote(v, ch);
+            }
           }
           ++acc_iter;
         }
