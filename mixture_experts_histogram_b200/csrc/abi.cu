@@ -127,7 +127,8 @@ struct Prof {
 };
 
 struct Maps {
-  CUtensorMap x, wr, xp, w1, w3, sw1, sw3, h, w2, sw2, w2h, sw2h;  // w2h/sw2h: 128-row boxes
+  CUtensorMap x, wr, w1, w3, sw1, sw3, w2, sw2, w2h, sw2h;  // w2h/sw2h: 128-row boxes
+  AMaps xp, h;                                           // GEMM1 / GEMM2 activations
 };
 
 void router_shape(int E, int* nbox, int* box_rows) {
@@ -251,10 +252,13 @@ int run_experts(const moe_config* c, const WsLayout& L, int64_t T, const void* x
   prof.mark();
 
   Maps m;
-  bool ok = map_2d(&m.xp, ws + L.xp, fp8, H, R, box_k, kTileM) &&
+  auto amaps = [&](AMaps* a, const void* base, uint64_t inner) {
+    return map_2d(&a->rows128, base, fp8, inner, R, box_k, 128) && map_2d(&a->rows64, base, fp8, inner, R, box_k, 64) &&
+           map_2d(&a->rows32, base, fp8, inner, R, box_k, 32);
+  };
+  bool ok = amaps(&m.xp, ws + L.xp, H) && amaps(&m.h, ws + L.h, I) &&
             map_2d(&m.w1, w->w1, fp8, H, (uint64_t)E * I, box_k, 128) &&
             map_2d(&m.w3, w->w3, fp8, H, (uint64_t)E * I, box_k, 128) &&
-            map_2d(&m.h, ws + L.h, fp8, I, R, box_k, kTileM) &&
             map_2d(&m.w2, w->w2, fp8, I, (uint64_t)E * H, box_k, 256) &&
             map_2d(&m.w2h, w->w2, fp8, I, (uint64_t)E * H, box_k, 128);
   if (S) {

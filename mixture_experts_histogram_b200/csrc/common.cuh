@@ -116,11 +116,20 @@ cudaError_t launch_scatter(const PermuteParams& p, cudaStream_t s);
 cudaError_t launch_gather(const GatherParams& p, bool fp8, cudaStream_t s);
 // pair: run the 2-SM (CTA pair, M = 256) variant; p.mt_prefix must then be the
 // pair-tile prefix and `grid` even.
-cudaError_t launch_gemm1(const GemmParams& p, bool fp8, bool pair, int grid, const CUtensorMap& tm_a,
+// Activation (A) tensor maps of one grouped GEMM: the same rows with 128-, 64-
+// and 32-row boxes. A tile loads the smallest box that covers its group's rows
+// (decode tiles hold one or two rows; a group's last tile is often short); the
+// MMA still reads 128 rows, and the rows past the box only feed output rows that
+// are never stored.
+struct AMaps {
+  CUtensorMap rows128, rows64, rows32;
+};
+
+cudaError_t launch_gemm1(const GemmParams& p, bool fp8, bool pair, int grid, const AMaps& tm_a,
                          const CUtensorMap& tm_w1, const CUtensorMap& tm_w3, const CUtensorMap& tm_sw1,
                          const CUtensorMap& tm_sw3, cudaStream_t s);
 // tm_w2 / tm_sw2 use 256-row boxes, tm_w2h / tm_sw2h the same tensors with 128-row boxes.
-cudaError_t launch_gemm2(const GemmParams& p, bool fp8, bool pair, int grid, const CUtensorMap& tm_a,
+cudaError_t launch_gemm2(const GemmParams& p, bool fp8, bool pair, int grid, const AMaps& tm_a,
                          const CUtensorMap& tm_w2, const CUtensorMap& tm_w2h, const CUtensorMap& tm_sw2,
                          const CUtensorMap& tm_sw2h, cudaStream_t s);
 cudaError_t launch_combine(const CombineParams& p, cudaStream_t s);

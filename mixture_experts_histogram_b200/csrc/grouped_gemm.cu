@@ -153,7 +153,7 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, int* s
 
 template <bool kFP8, bool kGemm1, bool kPair>
 __global__ void __launch_bounds__(kThreads, 1)
-    grouped_gemm_kernel(const GemmParams p, const __grid_constant__ CUtensorMap tm_a,
+    grouped_gemm_kernel(const GemmParams p, const __grid_constant__ AMaps tm_a,
                         const __grid_constant__ CUtensorMap tm_b0, const __grid_constant__ CUtensorMap tm_b1,
                         const __grid_constant__ CUtensorMap tm_bs0, const __grid_constant__ CUtensorMap tm_bs1) {
   using C = Cfg<kPair>;
@@ -205,7 +205,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     fence_mbar_init();
   }
   if (warp == 0 && lane == 0) {
-    tma_prefetch_desc(&tm_a);
+    tma_prefetch_desc(&tm_a.rows128);
+    tma_prefetch_desc(&tm_a.rows64);
+    tma_prefetch_desc(&tm_a.rows32);
     tma_prefetch_desc(&tm_b0);
     tma_prefetch_desc(&tm_bs0);
     tma_prefetch_desc(&tm_b1);
@@ -249,6 +251,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool shared = (it.g == p.E);
       const int my_row0 = it.row0 + my_off;
       const BRows<kGemm1> rows(it, p, &tm_b0, &tm_b1, &tm_bs0, &tm_bs1);
+      // A box: the smallest of 32 / 64 / 128 rows that covers this CTA's rows of
+      // the group (bytes per stage a_bytes; the pair leader also needs its peer's).
+      auto a_rows = [&](int row0) { const int v = it.end - row0; return v <= 32 ? 32 : (v <= 64 ? 64 : 128); };
+      const int my_a_rows = a_rows(my_row0);
+      const CUtensorMap* amap = my_a_rows == 32 ? &tm_a.rows32 : (my_a_rows == 64 ? &tm_a.rows64 : &tm_a.rows128);
+      const uint32_t stage_tx = kPair ? (uint32_t)(a_rows(it.row0) + a_rows(it.row0 + kTileM)) * kStageBytesK +
+                                            2u * C::kBBytes
+                                      : (uint32_t)my_a_rows * kStageBytesK + C::kBBytes;
       // FP8: where this tile's weight-block scales start (one fp32 per K block).
       const float *sb0 = nullptr, *sb1 = nullptr;
       if (kFP8) {
@@ -275,14 +285,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (kPair) {
             // Both CTAs' tiles complete on the even CTA's barrier, which expects them all.
             const uint32_t bar0 = map_to_cta(&full[stage], 0);
-            if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2 * C::kStageBytes);
-            tma_load_2d_pair(sA + stage * kABytes, &tm_a, bar0, kx, my_row0);
+            if (rank == 0) mbar_arrive_expect_tx(&full[stage], stage_tx);
+            tma_load_2d_pair(sA + stage * kABytes, amap, bar0, kx, my_row0);
             // GEMM2's 128-row halves come from the 128-row-box map (passed as the second map).
             tma_load_2d_pair(sB + stage * C::kBBytes, (kGemm1 && rank == 0) ? rows.m0 : rows.m1, bar0, kx,
                              rank ? rows.yb2 : rows.yb);
           } else {
-            mbar_arrive_expect_tx(&full[stage], C::kStageBytes);
-            tma_load_2d(sA + stage * kABytes, &tm_a, &full[stage], kx, my_row0);
+            mbar_arrive_expect_tx(&full[stage], stage_tx);
+            tma_load_2d(sA + stage * kABytes, amap, &full[stage], kx, my_row0);
             if (kGemm1) {
               tma_load_2d(sB + stage * C::kBBytes, rows.m0, &full[stage], kx, rows.yb);
               tma_load_2d(sB + stage * C::kBBytes + C::kBBytes / 2, rows.m1, &full[stage], kx, rows.yb2);
@@ -591,7 +601,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 template <bool kFP8, bool kGemm1, bool kPair>
-cudaError_t launch_one(const GemmParams& p, int grid, const CUtensorMap& a, const CUtensorMap& b0,
+cudaError_t launch_one(const GemmParams& p, int grid, const AMaps& a, const CUtensorMap& b0,
                        const CUtensorMap& b1, const CUtensorMap& bs0, const CUtensorMap& bs1, cudaStream_t s) {
   auto kern = grouped_gemm_kernel<kFP8, kGemm1, kPair>;
   static bool attr_set = false;  // per process; one device's limit serves every B200
@@ -622,7 +632,7 @@ cudaError_t launch_one(const GemmParams& p, int grid, const CUtensorMap& a, cons
 
 }  // namespace
 
-cudaError_t launch_gemm1(const GemmParams& p, bool fp8, bool pair, int grid, const CUtensorMap& tm_a,
+cudaError_t launch_gemm1(const GemmParams& p, bool fp8, bool pair, int grid, const AMaps& tm_a,
                          const CUtensorMap& tm_w1, const CUtensorMap& tm_w3, const CUtensorMap& tm_sw1,
                          const CUtensorMap& tm_sw3, cudaStream_t s) {
   if (pair)
@@ -632,7 +642,7 @@ cudaError_t launch_gemm1(const GemmParams& p, bool fp8, bool pair, int grid, con
              : launch_one<false, true, false>(p, grid, tm_a, tm_w1, tm_w3, tm_sw1, tm_sw3, s);
 }
 
-cudaError_t launch_gemm2(const GemmParams& p, bool fp8, bool pair, int grid, const CUtensorMap& tm_a,
+cudaError_t launch_gemm2(const GemmParams& p, bool fp8, bool pair, int grid, const AMaps& tm_a,
                          const CUtensorMap& tm_w2, const CUtensorMap& tm_w2h, const CUtensorMap& tm_sw2,
                          const CUtensorMap& tm_sw2h, cudaStream_t s) {
   if (pair)
