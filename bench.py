@@ -383,11 +383,16 @@ def traffic_for(kernel: str, workload_name: str):
         return None
 
 
+# Sources that build the grouped GEMM and its launch (tensor maps, variant
+# choice): the files a traffic figure for that kernel depends on.
+GEMM_SOURCES = ("grouped_gemm.cu", "ptx.cuh", "common.cuh", "abi.cu")
+
+
 def kernel_source_sha() -> str:
     import hashlib
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "mixture_experts_histogram_b200", "csrc")
-    for f in sorted(os.listdir(csrc)):
+    for f in GEMM_SOURCES:
         h.update(open(os.path.join(csrc, f), "rb").read())
     return h.hexdigest()[:16]
 
