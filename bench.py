@@ -418,7 +418,8 @@ def cpu_baseline(shape, x_np, w_np, target_s=12.0):
     """The oracle, as it stands, on all host cores, on a bounded token sample."""
     n = _pick_sample(shape, x_np, w_np, target_s)
     dt = _oracle_sample(shape, x_np, w_np, n)
-    return {"value": round(n / dt, 3), "unit": "tokens/s", "cores": os.cpu_count(), "kind": "oracle",
+    import oracle
+    return {"value": round(n / dt, 3), "unit": "tokens/s", "cores": oracle.num_threads(), "kind": "oracle",
             "sample": f"first {n} tokens of the workload: routing, experts and combine ({dt:.1f} s)"}
 
 
@@ -426,6 +427,7 @@ def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
+    import oracle
     import synth
     shape = workload(args.workload, args.tokens, args.experts)
     x_np = synth.make_x(shape)
@@ -442,7 +444,7 @@ def run_reference(args):
             "scaling": "weak", "vs_baseline": None, "dtype": "f64 accumulation (oracle)",
             "data": "synthetic (seeded, counter-based generator)", "impl": "reference",
             "config": describe(shape),
-            "cpu_baseline": {"value": round(value, 3), "unit": "tokens/s", "cores": os.cpu_count(),
+            "cpu_baseline": {"value": round(value, 3), "unit": "tokens/s", "cores": oracle.num_threads(),
                              "kind": "oracle", "sample": f"first {n} tokens of the workload per step"},
             "e2e": {"value": round(value, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)

@@ -59,6 +59,8 @@ def _load():
         build()
         lib = ctypes.CDLL(_SO)
         vp, i64, i32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32
+        lib.orc_num_threads.argtypes = []
+        lib.orc_num_threads.restype = ctypes.c_int
         lib.orc_e4m3_value.argtypes = [ctypes.c_uint8]
         lib.orc_e4m3_value.restype = ctypes.c_double
         lib.orc_e4m3_encode.argtypes = [ctypes.c_float]
@@ -83,6 +85,11 @@ def _p(a: Optional[np.ndarray]):
 
 
 # ------------------------------------------------------------------ E4M3 ----
+
+def num_threads() -> int:
+    """Threads the oracle's OpenMP loops use (reported beside its timings)."""
+    return int(_load().orc_num_threads())
+
 
 def e4m3_decode(codes: np.ndarray) -> np.ndarray:
     """Exact values (float64) of E4M3 codes (uint8)."""

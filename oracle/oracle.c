@@ -40,6 +40,9 @@
 #include <stdint.h>
 #include <stdlib.h>
 #include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
 
 /* ---------------------------------------------------------------- bf16 ---- */
 
@@ -88,6 +91,16 @@ static void e4m3_init(void) {
     E4M3_POS[c] = (e == 0) ? (float)m / 512.0f : ldexpf(1.0f + (float)m / 8.0f, e - 7);
   }
   e4m3_ready = 1;
+}
+
+/* Threads the OpenMP loops below run on (1 without OpenMP): reported with the
+ * oracle's timings. */
+int orc_num_threads(void) {
+#ifdef _OPENMP
+  return omp_get_max_threads();
+#else
+  return 1;
+#endif
 }
 
 double orc_e4m3_value(uint8_t c) {
