@@ -90,6 +90,12 @@ ROUTE_CASES = [
     synth.SWEEP_FP8.with_tokens(1),
     synth.MoeShape("wide-E512-k16", T=1000, hidden=512, n_experts=512, top_k=16, n_shared=1, inter=128, seed=9),
     synth.MoeShape("E300-k5", T=257, hidden=384, n_experts=300, top_k=5, n_shared=0, inter=128, seed=10),
+    # One full 128-token tile, one row past it, and a ragged skewed case (the K
+    # split changes with the number of token tiles).
+    synth.MoeShape("route-T128", T=128, hidden=4096, n_experts=352, top_k=8, n_shared=1, inter=1536, seed=26),
+    synth.MoeShape("route-T13-E300-skew", T=13, hidden=1024, n_experts=300, top_k=6, n_shared=0, inter=256,
+                   seed=27, skew=True),
+    synth.MoeShape("route-T129", T=129, hidden=4096, n_experts=352, top_k=8, n_shared=1, inter=1536, seed=28),
 ]
 
 
