@@ -188,33 +188,45 @@ __global__ void __launch_bounds__(256) topk_kernel(const TopkParams p) {
       if (p.logits) p.logits[t * p.E + e] = l[i];
     }
   }
-  uint32_t taken = 0;
+  // Selection on 64-bit keys: high word the logit's bits mapped to an unsigned
+  // order (larger logit, larger key), low word ~e (equal logits: the lower
+  // expert index wins). Each lane keeps the best of its own candidates; a round
+  // is one warp max, after which only the winning lane rescans its candidates.
+  uint64_t key[kPer];
+#pragma unroll
+  for (int i = 0; i < kPer; ++i) {
+    const int e = lane + 32 * i;
+    const uint32_t u = __float_as_uint(l[i] == 0.0f ? 0.0f : l[i]);  // -0 ties with +0, as floats do
+    const uint32_t ord = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+    key[i] = e < p.E ? ((uint64_t)ord << 32) | (uint32_t)~(uint32_t)e : 0ull;
+  }
+  uint64_t best = 0;
+#pragma unroll
+  for (int i = 0; i < kPer; ++i) best = key[i] > best ? key[i] : best;
+  uint32_t taken = 0;  // bit i: candidate i of this lane already chosen
   float my_v = -INFINITY;
   int my_e = 0;
   for (int j = 0; j < p.k; ++j) {
-    float bv = -INFINITY;
-    int be = 0x7FFFFFFF;
-#pragma unroll
-    for (int i = 0; i < kPer; ++i) {
-      const int e = lane + 32 * i;
-      if (e < p.E && !(taken & (1u << i)) && (l[i] > bv || (l[i] == bv && e < be))) {
-        bv = l[i];
-        be = e;
-      }
-    }
+    uint64_t top = best;
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) {
-      const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
-      const int oe = __shfl_xor_sync(0xffffffffu, be, off);
-      if (ov > bv || (ov == bv && oe < be)) {
-        bv = ov;
-        be = oe;
+      const uint64_t o = __shfl_xor_sync(0xffffffffu, top, off);
+      top = o > top ? o : top;
+    }
+    const int e = (int)~(uint32_t)top;
+    if ((e & 31) == lane) {
+      taken |= 1u << (e >> 5);
+      best = 0;
+#pragma unroll
+      for (int i = 0; i < kPer; ++i) {
+        const uint64_t kk = (taken >> i) & 1u ? 0ull : key[i];
+        best = kk > best ? kk : best;
       }
     }
-    if ((be & 31) == lane) taken |= 1u << (be >> 5);
     if (lane == j) {
-      my_v = bv;
-      my_e = be;
+      const uint32_t ord = (uint32_t)(top >> 32);
+      my_v = __uint_as_float((ord & 0x80000000u) ? (ord & 0x7FFFFFFFu) : ~ord);
+      my_e = e;
     }
   }
   const float m = __shfl_sync(0xffffffffu, my_v, 0);
