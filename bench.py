@@ -42,7 +42,8 @@ def parse_args():
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=["prefill-fp8", "decode-bf16", "long-skew-fp8"], default="prefill-fp8")
+    ap.add_argument("--workload", choices=["prefill-fp8", "decode-bf16", "long-skew-fp8", "dense-ffn-fp8"],
+                    default="prefill-fp8")
     ap.add_argument("--no-decode", action="store_true", help="skip the T=64 FP8 decode line")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
@@ -55,7 +56,7 @@ def workload(name, tokens=None, experts=None):
     import dataclasses
     import synth
     s = {"prefill-fp8": synth.PREFILL_FP8, "decode-bf16": synth.DECODE_BF16,
-         "long-skew-fp8": synth.LONG_SKEW_FP8}[name]
+         "long-skew-fp8": synth.LONG_SKEW_FP8, "dense-ffn-fp8": synth.DENSE_FFN_FP8}[name]
     if experts is not None:
         s = dataclasses.replace(s, n_experts=experts, name=f"{s.name}-E{experts}")
     if tokens is not None:
@@ -279,7 +280,7 @@ def run_ours(args):
             dshape = shape.with_tokens(64)
             decode = measure(64, synth.make_x(dshape), e2e=False)
     decode_bf16 = None
-    if not args.no_decode and shape.wdtype == synth.WDTYPE_FP8:
+    if not args.no_decode and shape.wdtype == synth.WDTYPE_FP8 and args.workload == "prefill-fp8":
         # The BF16 decode workload (its own seed and BF16 weights).
         del wd, wts
         torch.cuda.empty_cache()

@@ -147,8 +147,12 @@ PREFILL_FP8 = MoeShape("step5-prefill-fp8", T=8192, wdtype=WDTYPE_FP8, seed=2)
 LONG_SKEW_FP8 = MoeShape("step5-long-prefill-zipf-fp8", T=32768, wdtype=WDTYPE_FP8, seed=3, skew=True)
 SWEEP_FP8 = MoeShape("step5-decode-sweep-fp8", T=64, wdtype=WDTYPE_FP8, seed=4)
 SWEEP_TOKENS = (1, 8, 64, 512, 2048)
+# The dense SwiGLU FFN of layers 0-2 and 91 (intermediate 13,824): the same layer
+# with one expert, top-1 routing (gate 1) and no shared expert.
+DENSE_FFN_FP8 = MoeShape("step5-dense-ffn-fp8", T=8192, n_experts=1, top_k=1, n_shared=0, inter=13824,
+                         wdtype=WDTYPE_FP8, seed=5)
 
-WORKLOADS = {w.name: w for w in (TINY, DECODE_BF16, PREFILL_FP8, LONG_SKEW_FP8, SWEEP_FP8)}
+WORKLOADS = {w.name: w for w in (TINY, DECODE_BF16, PREFILL_FP8, LONG_SKEW_FP8, SWEEP_FP8, DENSE_FFN_FP8)}
 
 
 def zipf_bias(seed: int, E: int, alpha: float = ZIPF_ALPHA) -> np.ndarray:

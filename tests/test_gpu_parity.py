@@ -307,6 +307,10 @@ def _layer_cases():
                         wdtype=synth.WDTYPE_FP8, seed=24), None),
         (synth.MoeShape("auto-pair-bf16", T=520, hidden=384, n_experts=6, top_k=2, n_shared=0, inter=384,
                         seed=25), None),
+        # The dense SwiGLU FFN (one expert, top-1, no shared expert, I = 13,824).
+        (synth.DENSE_FFN_FP8.with_tokens(300), 12),
+        (dataclasses.replace(synth.DENSE_FFN_FP8, name="step5-dense-ffn-bf16", wdtype=synth.WDTYPE_BF16)
+         .with_tokens(64), 8),
         (synth.DECODE_BF16, None),
         (synth.SWEEP_FP8.with_tokens(1), None),
         (synth.SWEEP_FP8.with_tokens(8), None),
