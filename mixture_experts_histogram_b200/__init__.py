@@ -96,7 +96,8 @@ def _ptr(t) -> Optional[int]:
     if isinstance(t, int):
         return t
     if hasattr(t, "data_ptr"):
-        assert t.is_contiguous(), "tensors passed to the library must be contiguous"
+        if not t.is_contiguous():
+            raise ValueError("tensors passed to the library must be contiguous")
         return t.data_ptr()
     return t.ctypes.data  # numpy
 
