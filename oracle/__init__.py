@@ -17,6 +17,11 @@ Functions and the passages they follow:
                    slot order (README, "Long-output stability": fixed-order
                    accumulation in at least fp32)
   moe_forward      route + moe_tokens for a whole batch (or a token sample)
+  rmsnorm          the fp32 residual stream normalised into the layer's bf16
+                   input (NeMo "Step-5-Preview" page, "Full-Depth H100
+                   Benchmark" table: FP32 norms and residuals)
+  add_residual     the layer output added back into the fp32 residual stream
+                   (same table; "Attention and Precision": FP32 residual stream)
 """
 from __future__ import annotations
 
@@ -199,3 +204,29 @@ def moe_forward(shape, weights: dict, x_bf16: np.ndarray, tokens: Optional[Seque
                               want_logits=True)
     out, outb, _ = moe_tokens(shape, weights, x_bf16, idx, gate, tokens)
     return {"idx": idx, "gate": gate, "logits": logits, "out_f64": out, "out_bf16": outb}
+
+
+# ---------------------------------------------------------- residual stream --
+
+def rmsnorm(residual: np.ndarray, weight: np.ndarray, eps: float) -> np.ndarray:
+    """y = r / sqrt(mean(r^2) + eps) * w per row, in fp64 (r: [T, H] fp32, w: [H]).
+
+    The pages fix only that norms are fp32; the norm type (RMS, no mean
+    subtraction, no bias) and eps follow the usual decoder reading.
+    """
+    r = residual.astype(np.float64)
+    ms = np.mean(r * r, axis=1, keepdims=True)
+    return r / np.sqrt(ms + eps) * weight.astype(np.float64)[None, :]
+
+
+def add_residual(residual: np.ndarray, y_rows: np.ndarray, pos: np.ndarray) -> np.ndarray:
+    """r_out[t] = r[t] + sum_j y[pos[t, j]] in fp64 (slots in order; pos < 0 skipped)."""
+    out = residual.astype(np.float64).copy()
+    T, S = pos.shape
+    for t in range(T):
+        acc = np.zeros(residual.shape[1], np.float64)
+        for j in range(S):
+            if pos[t, j] >= 0:
+                acc += y_rows[pos[t, j]].astype(np.float64)
+        out[t] += acc
+    return out

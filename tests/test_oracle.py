@@ -312,3 +312,40 @@ def test_zipf_skew_gives_about_ten_times_the_mean_load():
     cnt = np.bincount(idx.ravel(), minlength=shape.n_experts)
     ratio = cnt.max() / cnt.mean()
     assert 8.0 <= ratio <= 12.5, ratio
+
+
+# ------------------------------------------------------------ residual stream --
+
+def test_rmsnorm_closed_forms():
+    H, eps = 256, 1e-6
+    w = np.linspace(0.5, 1.5, H)
+    # A constant row c: every element is c / sqrt(c^2 + eps) * w.
+    r = np.full((1, H), 3.0, np.float32)
+    np.testing.assert_allclose(oracle.rmsnorm(r, w, eps)[0], 3.0 / np.sqrt(9.0 + eps) * w, rtol=1e-14)
+    # One non-zero element a: mean(r^2) = a^2 / H.
+    r = np.zeros((1, H), np.float32)
+    r[0, 7] = -2.0
+    y = oracle.rmsnorm(r, w, eps)[0]
+    assert y[7] == pytest.approx(-2.0 / np.sqrt(4.0 / H + eps) * w[7], rel=1e-14)
+    assert np.count_nonzero(y) == 1
+
+
+def test_rmsnorm_is_scale_invariant_and_unit_rms():
+    rng = np.random.default_rng(3)
+    r = rng.standard_normal((5, 384)).astype(np.float32)
+    ones = np.ones(384)
+    y1 = oracle.rmsnorm(r, ones, 0.0)
+    y2 = oracle.rmsnorm(np.float32(8.0) * r, ones, 0.0)
+    np.testing.assert_allclose(y1, y2, rtol=1e-12)
+    np.testing.assert_allclose(np.sqrt(np.mean(y1 * y1, axis=1)), 1.0, rtol=1e-12)
+
+
+def test_add_residual_sums_slots_and_skips_negative_positions():
+    rng = np.random.default_rng(4)
+    r = rng.standard_normal((3, 8)).astype(np.float32)
+    y = rng.standard_normal((6, 8)).astype(np.float32)
+    pos = np.array([[0, 1], [2, -1], [5, 4]], np.int32)
+    out = oracle.add_residual(r, y, pos)
+    np.testing.assert_allclose(out[0], r[0].astype(np.float64) + y[0] + y[1], rtol=1e-14)
+    np.testing.assert_allclose(out[1], r[1].astype(np.float64) + y[2], rtol=1e-14)
+    np.testing.assert_allclose(out[2], r[2].astype(np.float64) + y[5] + y[4], rtol=1e-14)
