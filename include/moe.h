@@ -192,6 +192,26 @@ MOE_API int moe_experts(const moe_config* cfg, int64_t T, const void* x, const i
 MOE_API int moe_combine(const moe_config* cfg, int64_t T, const void* y, const int32_t* pos, void* out,
                 moe_stream_t stream);
 
+/* ---- the fp32 residual stream around the layer ----
+ * (NeMo "Step-5-Preview" page, "Full-Depth H100 Benchmark" table: FP32 norms and
+ * residuals.) The norm's type is not stated there; these follow the usual
+ * decoder reading: RMS normalisation without mean subtraction or bias. */
+
+/* x[t] = bf16(r[t] / sqrt(mean_h(r[t, h]^2) + eps) * weight), computed in fp32
+ * (IEEE sqrt and division), rounded once to bf16: the layer's input.
+ * residual [T, H] fp32, weight [H] fp32, x_bf16 [T, H] bf16 (device, 16-byte
+ * aligned); H a multiple of 128; eps >= 0. */
+MOE_API int moe_rmsnorm(int64_t T, int32_t hidden, const float* residual, const float* weight, float eps,
+                void* x_bf16, moe_stream_t stream);
+
+/* The combine with the residual add: r_out[t] = r[t] + sum over slots j of
+ * y[pos[t, j]], the rows summed in fp32 in slot order and added to r in fp32
+ * (no bf16 rounding of the layer output). y and pos as for moe_combine (rows
+ * with pos < 0 are skipped); residual, residual_out [T, H] fp32, which may be
+ * the same buffer. */
+MOE_API int moe_combine_residual(const moe_config* cfg, int64_t T, const void* y, const int32_t* pos,
+                const float* residual, float* residual_out, moe_stream_t stream);
+
 /* ---- status and profiling ---- */
 
 /* Synchronises `stream`, then returns the device status latched in the

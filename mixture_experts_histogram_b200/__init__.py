@@ -9,7 +9,7 @@ The functions carry the names of the C entry points:
   moe_workspace_bytes, moe_forward, moe_forward_host, moe_route,
   moe_quantize_act, moe_permute, moe_experts, moe_combine, moe_read_status,
   moe_status_string, moe_profile_enable, moe_profile_read, moe_device_sm_count,
-  moe_set_gemm_variant, moe_permute_noalloc.
+  moe_set_gemm_variant, moe_permute_noalloc, moe_rmsnorm, moe_combine_residual.
 """
 from __future__ import annotations
 
@@ -80,6 +80,8 @@ def load():
         "moe_device_sm_count": [ctypes.POINTER(ctypes.c_int)],
         "moe_set_gemm_variant": [ctypes.c_int],
         "moe_permute_noalloc": [cfgp, i64, vp, vp, vp, vp, vp, vp, vp],
+        "moe_rmsnorm": [i64, i32, vp, vp, ctypes.c_float, vp, vp],
+        "moe_combine_residual": [cfgp, i64, vp, vp, vp, vp, vp],
     }
     for name, args in sig.items():
         f = getattr(lib, name)
@@ -178,6 +180,18 @@ def moe_experts(cfg, T, x, topk_idx, topk_w, w: moe_weights, y, pos, workspace, 
 def moe_combine(cfg, T, y, pos, out, stream=None):
     _check(load().moe_combine(ctypes.byref(cfg), T, _ptr(y), _ptr(pos), _ptr(out), _stream(stream)),
            "moe_combine")
+
+
+def moe_rmsnorm(T, hidden, residual, weight, eps, x, stream=None):
+    """x = bf16(RMS-normalised fp32 residual * weight): the layer's input."""
+    _check(load().moe_rmsnorm(T, hidden, _ptr(residual), _ptr(weight), float(eps), _ptr(x), _stream(stream)),
+           "moe_rmsnorm")
+
+
+def moe_combine_residual(cfg, T, y, pos, residual, residual_out, stream=None):
+    """residual_out = residual + fixed-order fp32 sum of the token's expert rows."""
+    _check(load().moe_combine_residual(ctypes.byref(cfg), T, _ptr(y), _ptr(pos), _ptr(residual),
+                                       _ptr(residual_out), _stream(stream)), "moe_combine_residual")
 
 
 def moe_read_status(workspace, stream=None) -> int:

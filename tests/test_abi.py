@@ -87,6 +87,24 @@ def test_argument_errors_need_no_device(lib):
         m.MOE_OK
 
 
+def test_residual_stream_argument_errors_need_no_device(lib):
+    # moe_rmsnorm(T, hidden, residual, weight, eps, x, stream)
+    # (Every call below returns before any launch: these are host addresses.)
+    assert lib.moe_rmsnorm(4, 100, 1024, 2048, 1e-6, 4096, None) == m.MOE_ERR_INVALID_ARG   # H not a multiple of 128
+    assert lib.moe_rmsnorm(4, 256, 1024, 2048, -1.0, 4096, None) == m.MOE_ERR_INVALID_ARG   # negative eps
+    assert lib.moe_rmsnorm(-1, 256, 1024, 2048, 1e-6, 4096, None) == m.MOE_ERR_INVALID_ARG
+    assert lib.moe_rmsnorm(4, 256, None, 2048, 1e-6, 4096, None) == m.MOE_ERR_INVALID_ARG
+    assert lib.moe_rmsnorm(4, 256, 1028, 2048, 1e-6, 4096, None) == m.MOE_ERR_MISALIGNED
+    assert lib.moe_rmsnorm(0, 256, None, None, 1e-6, None, None) == m.MOE_OK               # T = 0: no-op
+    # moe_combine_residual(cfg, T, y, pos, residual, residual_out, stream)
+    cfg = m.make_config(256, 16, 2, 1, 128, 0)
+    assert lib.moe_combine_residual(ctypes.byref(cfg), 4, 1024, 2048, 4096, 8192 + 4, None) == m.MOE_ERR_MISALIGNED
+    assert lib.moe_combine_residual(ctypes.byref(cfg), 4, 1024, None, 4096, 8192, None) == m.MOE_ERR_INVALID_ARG
+    bad = m.make_config(200, 16, 2, 1, 128, 0)
+    assert lib.moe_combine_residual(ctypes.byref(bad), 4, 1024, 2048, 4096, 8192, None) == m.MOE_ERR_INVALID_ARG
+    assert lib.moe_combine_residual(ctypes.byref(cfg), 0, None, None, None, None, None) == m.MOE_OK
+
+
 def test_status_strings(lib):
     for c in range(8):
         assert m.moe_status_string(c) not in ("", "unknown status")
