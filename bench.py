@@ -47,6 +47,8 @@ def parse_args():
     ap.add_argument("--no-decode", action="store_true", help="skip the T=64 FP8 decode line")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--residual", action="store_true",
+                    help="also time the residual-stream kernels (RMSNorm in, residual combine out)")
     ap.add_argument("--tokens", type=int, default=None, help="override T (profiling cases)")
     ap.add_argument("--experts", type=int, default=None, help="override E (profiling cases)")
     return ap.parse_args()
@@ -361,6 +363,8 @@ def run_ours(args):
                                    "layer_roofline": blayer,
                                    "kernel_ms": {k: round(v, 4) for k, v in bres["kernel_ms"].items()},
                                    "config": describe(bshape)}
+    if args.residual:
+        line["residual_stream"] = time_residual(m, shape, args, pk, local, flush)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(shape, x_np, w_np)
     if rank == 0:
@@ -368,6 +372,46 @@ def run_ours(args):
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
+
+
+def time_residual(m, shape, args, pk, local, flush):
+    """moe_rmsnorm and moe_combine_residual at the workload's T, against measured HBM.
+
+    Algorithmic bytes: RMSNorm reads r (4TH) and w (4H), writes x (2TH); the
+    residual combine reads the (k+S)T expert rows (2H each) and r, writes r_out.
+    """
+    import numpy as np
+    import torch
+    T, H, k, S = shape.T, shape.hidden, shape.top_k, shape.n_shared
+    dev = f"cuda:{local}"
+    g = torch.Generator(device=dev).manual_seed(shape.seed)
+    r = torch.randn((T, H), generator=g, device=dev, dtype=torch.float32)
+    w = torch.ones(H, device=dev, dtype=torch.float32)
+    x = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
+    rows = (k + S) * T
+    y = torch.randn((rows, H), generator=g, device=dev, dtype=torch.float32).to(torch.bfloat16)
+    pos = torch.randperm(rows, generator=g, device=dev).to(torch.int32).view(T, k + S)
+    r_out = torch.empty_like(r)
+    cfg = m.make_config(H, shape.n_experts, k, S, shape.inter, shape.wdtype)
+    res = {}
+    for name, fn, nbytes in (
+            ("rmsnorm", lambda: m.moe_rmsnorm(T, H, r, w, 1e-6, x), 4 * T * H + 4 * H + 2 * T * H),
+            ("combine_residual", lambda: m.moe_combine_residual(cfg, T, y, pos, r, r_out),
+             2 * rows * H + 4 * T * H + 4 * T * H)):
+        for _ in range(max(args.warmup, 3)):
+            fn()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+        for i in range(args.steps):
+            flush.fill_(i & 0xFF)
+            ev[i][0].record()
+            fn()
+            ev[i][1].record()
+        torch.cuda.synchronize()
+        ms = float(np.mean([a.elapsed_time(b) for a, b in ev]))
+        gbs = nbytes / (ms / 1e3) / 1e9
+        res[name] = {"ms": round(ms, 4), "algorithmic_bytes": nbytes, "achieved_gbs": round(gbs, 1),
+                     "frac_of_hbm": round(gbs / pk["hbm_gbs"], 4)}
+    return res
 
 
 def traffic_for(kernel: str, workload_name: str):
