@@ -45,6 +45,8 @@ def parse_args():
     ap.add_argument("--workload", choices=["prefill-fp8", "decode-bf16", "long-skew-fp8", "dense-ffn-fp8"],
                     default="prefill-fp8")
     ap.add_argument("--no-decode", action="store_true", help="skip the T=64 FP8 decode line")
+    ap.add_argument("--no-extra", action="store_true",
+                    help="skip the Zipf-skewed T=32768 long prefill and the FP8 decode-sweep lines")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--residual", action="store_true",
@@ -227,6 +229,7 @@ def run_ours(args):
         if world > 1:
             dist.barrier()
         torch.cuda.synchronize()
+        launches0 = m.moe_launch_count()
         # Timed steps: no per-kernel events inside. Before each step ~1 ms of GPU
         # sleep (outside ev0..ev1) lets the host queue the whole step, so the
         # device time is not stretched by host launch gaps.
@@ -237,6 +240,7 @@ def run_ours(args):
             step()
             ev[i][1].record(stream)
         torch.cuda.synchronize()
+        launches = m.moe_launch_count() - launches0
         if world > 1:
             dist.barrier()
         total_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in ev), world, f"cuda:{local}")
@@ -256,22 +260,47 @@ def run_ours(args):
             raise RuntimeError(f"device status after timing: {m.moe_status_string(st)}")
         res = {"ms_per_step": total_ms / args.steps, "tokens_per_s": replica_throughput(T, world, args.steps, total_ms),
                "kernel_ms": {k: v / args.steps for k, v in per_kernel.items()},
-               "idx": idx.cpu().numpy()}
+               "idx": idx.cpu().numpy(), "launches": launches}
         if e2e:
+            # End to end through the host-buffer entry points: every step copies
+            # its x in from pinned host memory and its output back out.
             xh = torch.from_numpy(np.ascontiguousarray(x_host).view(np.int16)).pin_memory()
-            oh = torch.empty((T, shape.hidden), dtype=torch.int16).pin_memory()
+            oh = [torch.empty((T, shape.hidden), dtype=torch.int16).pin_memory() for _ in range(2)]
             for _ in range(2):
-                m.moe_forward_host(cfg, T, xh, wts, oh, ws, stream=stream)
+                m.moe_forward_host(cfg, T, xh, wts, oh[0], ws, stream=stream)
+            # (a) one step at a time (moe_forward_host: copy in, layer, copy out, sync).
             ms = []
             for i in range(args.steps):
                 flush.fill_(i & 0xFF)
                 torch.cuda.synchronize()
                 t0 = time.perf_counter()
-                m.moe_forward_host(cfg, T, xh, wts, oh, ws, stream=stream)
+                m.moe_forward_host(cfg, T, xh, wts, oh[0], ws, stream=stream)
                 ms.append((time.perf_counter() - t0) * 1e3)
-            e2e_ms = max_over_ranks(sum(ms), world, f"cuda:{local}")
-            res["e2e"] = {"value": replica_throughput(T, world, args.steps, e2e_ms), "unit": "tokens/s",
-                          "h2d_bytes_per_step": T * shape.hidden * 2, "d2h_bytes_per_step": T * shape.hidden * 2}
+            serial_ms = max_over_ranks(sum(ms), world, f"cuda:{local}")
+            # (b) steps pipelined over two streams and two workspaces
+            # (moe_forward_host_async): one step's copies overlap the other's kernels.
+            ws2 = torch.empty_like(ws)
+            streams = [stream, torch.cuda.Stream(device=f"cuda:{local}")]
+            wss = [ws, ws2]
+            for i in range(4):
+                m.moe_forward_host_async(cfg, T, xh, wts, oh[i % 2], wss[i % 2], stream=streams[i % 2])
+            torch.cuda.synchronize()
+            t0 = time.perf_counter()
+            for i in range(args.steps):
+                m.moe_forward_host_async(cfg, T, xh, wts, oh[i % 2], wss[i % 2], stream=streams[i % 2])
+            torch.cuda.synchronize()
+            pipe_ms = max_over_ranks((time.perf_counter() - t0) * 1e3, world, f"cuda:{local}")
+            for wsx in wss:
+                st = m.moe_read_status(wsx)
+                if st != 0:
+                    raise RuntimeError(f"device status after the host-buffer steps: {m.moe_status_string(st)}")
+            del ws2
+            res["e2e"] = {"value": replica_throughput(T, world, args.steps, pipe_ms), "unit": "tokens/s",
+                          "h2d_bytes_per_step": T * shape.hidden * 2, "d2h_bytes_per_step": T * shape.hidden * 2,
+                          "how": "moe_forward_host_async, steps alternating two streams and workspaces, "
+                                 "host wall clock from the first copy in to the last copy out",
+                          "serial_value": replica_throughput(T, world, args.steps, serial_ms),
+                          "serial_how": "moe_forward_host, one synchronous step at a time, L2 flushed between"}
         return res
 
     pk = peaks()
@@ -284,7 +313,7 @@ def run_ours(args):
     decode_bf16 = None
     if not args.no_decode and shape.wdtype == synth.WDTYPE_FP8 and args.workload == "prefill-fp8":
         # The BF16 decode workload (its own seed and BF16 weights).
-        del wd, wts
+        wd = wts = None
         torch.cuda.empty_cache()
         bshape = synth.DECODE_BF16
         bw = m.upload_weights(synth.make_weights(bshape), f"cuda:{local}")
@@ -292,6 +321,21 @@ def run_ours(args):
             decode_bf16 = (bshape, measure(bshape.T, synth.make_x(bshape), e2e=False, shape=bshape,
                                            wts=m.make_weights(bw)))
         del bw
+    extra = {}
+    if not args.no_extra and args.workload == "prefill-fp8" and args.tokens is None and args.experts is None:
+        # The long skewed prefill and the FP8 decode sweep, each on its own
+        # seeded weights (freed between workloads).
+        for key, wshape, tokens in (("long_skew_t32768", synth.LONG_SKEW_FP8, [synth.LONG_SKEW_FP8.T]),
+                                    ("decode_sweep_fp8", synth.SWEEP_FP8, list(synth.SWEEP_TOKENS))):
+            wd = wts = None
+            torch.cuda.empty_cache()
+            ew = m.upload_weights(synth.make_weights(wshape), f"cuda:{local}")
+            ewts = m.make_weights(ew)
+            with ClockSampler(local) as eclk:
+                runs = [(T, measure(T, synth.make_x(wshape.with_tokens(T)), e2e=False, shape=wshape.with_tokens(T),
+                                    wts=ewts)) for T in tokens]
+            extra[key] = (wshape, runs, eclk.summary())
+            del ew, ewts
     clocks = clk.summary()
 
     def roofline(res, T, shape=shape):
@@ -311,6 +355,14 @@ def run_ours(args):
             "gemm2_down": {"bytes": groups * (H * I * es + scale2) + R * I * es + R * H * 2,
                            "flops": 2.0 * R * I * H},
         }
+        for kk, v in kern.items():
+            kms = res["kernel_ms"].get(kk, 0.0)
+            if kms > 0:
+                v["ms"] = round(kms, 4)
+                v["hbm_gbs"] = round(v["bytes"] / (kms / 1e3) / 1e9, 1)
+                v["hbm_frac"] = round(v["hbm_gbs"] / pk["hbm_gbs"], 4)
+                v["tflops"] = round(v["flops"] / (kms / 1e3) / 1e12, 1)
+                v["tensor_frac"] = round(v["tflops"] / (pk["fp8_tflops"] if shape.wdtype else pk["bf16_tflops"]), 4)
         dom = max(kern, key=lambda kk: res["kernel_ms"].get(kk, 0.0))
         ms = res["kernel_ms"][dom]
         t_hbm = kern[dom]["bytes"] / (pk["hbm_gbs"] * 1e9)
@@ -332,6 +384,8 @@ def run_ours(args):
         lay_flops = 2.0 * T * H * E + 2.0 * 3 * H * I * R
         t_roof = max(lay_bytes / (pk["hbm_gbs"] * 1e9), lay_flops / (peak_tf * 1e12))
         layer = {"ms": round(res["ms_per_step"], 4), "roofline_ms": round(t_roof * 1e3, 4),
+                 "expert_gemms": {kk: {q: v[q] for q in ("ms", "hbm_gbs", "hbm_frac", "tflops", "tensor_frac")
+                                       if q in v} for kk, v in kern.items()},
                  "frac": round(t_roof * 1e3 / res["ms_per_step"], 4),
                  "tflops": round(lay_flops / (res["ms_per_step"] / 1e3) / 1e12, 1),
                  "hbm_gbs_of_algorithmic_bytes": round(lay_bytes / (res["ms_per_step"] / 1e3) / 1e9, 1)}
@@ -346,7 +400,7 @@ def run_ours(args):
         "config": dict(describe(shape), parallelism=f"replicas x{world}" if world > 1 else "single GPU"),
         "roofline": roof, "layer_roofline": layer,
         "kernel_ms": {k: round(v, 4) for k, v in main["kernel_ms"].items()},
-        "e2e": main.get("e2e"), "gpu_launches": len(KERNELS) * args.steps, "clocks": clocks,
+        "e2e": main.get("e2e"), "gpu_launches": main["launches"], "clocks": clocks,
     }
     if decode is not None:
         droof, dlayer = roofline(decode, 64)
@@ -363,6 +417,19 @@ def run_ours(args):
                                    "layer_roofline": blayer,
                                    "kernel_ms": {k: round(v, 4) for k, v in bres["kernel_ms"].items()},
                                    "config": describe(bshape)}
+    for key, (wshape, runs, eclk) in extra.items():
+        sub = {}
+        for T, res in runs:
+            r_, l_ = roofline(res, T, shape=wshape.with_tokens(T))
+            counts = np.bincount(res["idx"].reshape(-1), minlength=wshape.n_experts)
+            sub[f"T={T}"] = {"value": round(res["tokens_per_s"], 1), "unit": "tokens/s",
+                             "ms_per_step": round(res["ms_per_step"], 4), "roofline": r_, "layer_roofline": l_,
+                             "kernel_ms": {k: round(v, 4) for k, v in res["kernel_ms"].items()},
+                             "routed_rows_per_expert": {"hottest": int(counts.max()),
+                                                        "mean": round(float(counts.mean()), 1),
+                                                        "hottest_over_mean": round(float(counts.max() / counts.mean()), 2)},
+                             "gpu_launches": res["launches"]}
+        line[key] = {"config": describe(wshape), "tokens": [T for T, _ in runs], "clocks": eclk, **sub}
     if args.residual:
         line["residual_stream"] = time_residual(m, shape, args, pk, local, flush)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -431,7 +498,7 @@ def traffic_for(kernel: str, workload_name: str):
 
 # Sources that build the grouped GEMM and its launch (tensor maps, variant
 # choice): the files a traffic figure for that kernel depends on.
-GEMM_SOURCES = ("grouped_gemm.cu", "ptx.cuh", "common.cuh", "abi.cu")
+GEMM_SOURCES = ("grouped_gemm.cu", "gemm_common.cuh", "ptx.cuh", "common.cuh", "abi.cu")
 
 
 def kernel_source_sha() -> str:
@@ -489,7 +556,7 @@ def run_reference(args):
             "warmup": warm, "ms_per_step": round(1e3 * sum(ts) / steps, 2), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64 accumulation (oracle)",
             "data": "synthetic (seeded, counter-based generator)", "impl": "reference",
-            "config": describe(shape),
+            "config": dict(describe(shape), parallelism="single GPU" if args.gpus <= 1 else f"replicas x{args.gpus}"),
             "cpu_baseline": {"value": round(value, 3), "unit": "tokens/s", "cores": oracle.num_threads(),
                              "kind": "oracle", "sample": f"first {n} tokens of the workload per step"},
             "e2e": {"value": round(value, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}

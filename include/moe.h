@@ -29,8 +29,10 @@
  *      the shared expert's sw1, sw3, sw2 (and ss1, ss3, ss2) have the same
  *      layouts with E = 1.
  *  - "Device" pointers are CUDA device memory of the current device; the
- *    caller owns every buffer. The library allocates no device memory: all
- *    scratch comes from the caller's workspace (size: moe_workspace_bytes).
+ *    caller owns every buffer. The library allocates no device memory per
+ *    call: all scratch comes from the caller's workspace (size:
+ *    moe_workspace_bytes), except moe_permute_noalloc's fixed 1 MiB
+ *    file-scope device array, which every GPU that loads the library holds.
  *  - Calls are asynchronous on `stream` unless stated. Argument errors are
  *    returned synchronously; errors found on the device (a bad expert index,
  *    a timed-out wait) are latched in a status word inside the workspace and
@@ -63,7 +65,8 @@ typedef struct CUstream_st* moe_stream_t;
 /* Expert weight storage. */
 enum {
   MOE_WDTYPE_BF16 = 0,     /* bf16 weights, bf16 activations */
-  MOE_WDTYPE_FP8_E4M3 = 1  /* E4M3 weights with 128x128 fp32 block scales, E4M3 1x128 activations */
+  MOE_WDTYPE_FP8_E4M3 = 1, /* E4M3 weights with 128x128 fp32 block scales, E4M3 1x128 activations */
+  MOE_WDTYPE_NVFP4 = 2     /* NVFP4 weights, bf16 activations (W4A16; see moe_weights) */
 };
 
 /* Status codes (returned, or latched on the device). */
@@ -88,8 +91,17 @@ typedef struct moe_config {
 } moe_config;
 
 /* Device pointers to one layer's weights (see the layouts above). Scale
- * pointers are used only for MOE_WDTYPE_FP8_E4M3; shared-expert pointers only
- * when n_shared == 1. router_bias may be NULL (no bias). */
+ * pointers are used only for MOE_WDTYPE_FP8_E4M3 and MOE_WDTYPE_NVFP4;
+ * shared-expert pointers only when n_shared == 1. router_bias may be NULL (no
+ * bias).
+ * MOE_WDTYPE_NVFP4 (TensorFold PR page: the NVFP4 format its W4A16 linears
+ * read; a variant the pages describe for another model): every expert matrix
+ * [n, k] is stored as E2M1 codes [n, k/2] uint8, two per byte with input 2j in
+ * the low nibble of byte j (w1/w3/w2 point to them), E4M3 scales [n, k/16]
+ * uint8, one per 16 inputs (s1/s3/s2), and one fp32 global scale per matrix
+ * (g1/g3/g2 [E]; the shared expert's sg1/sg3/sg2 [1]); an element is
+ * e2m1 x e4m3 x global. Activations and h stay bf16. Needs H and I multiples
+ * of 256. */
 typedef struct moe_weights {
   const void* router_w;
   const float* router_bias;
@@ -105,6 +117,12 @@ typedef struct moe_weights {
   const float* ss1;
   const float* ss3;
   const float* ss2;
+  const float* g1; /* NVFP4 global scales [E] */
+  const float* g3;
+  const float* g2;
+  const float* sg1; /* NVFP4 global scales of the shared expert [1] */
+  const float* sg3;
+  const float* sg2;
 } moe_weights;
 
 /* Bytes of workspace that moe_forward (and every stage entry point) needs for
@@ -131,6 +149,17 @@ MOE_API int moe_forward(const moe_config* cfg, int64_t T, const void* x, const m
  */
 MOE_API int moe_forward_host(const moe_config* cfg, int64_t T, const void* x_host, const moe_weights* w,
                      void* out_host, void* workspace, size_t workspace_bytes, moe_stream_t stream);
+
+/*
+ * moe_forward_host without the final synchronisation: the copy in, the layer
+ * and the copy out are queued on `stream` and the call returns. x_host and
+ * out_host must stay valid (and should be pinned) until the stream has passed
+ * the copy out (cudaStreamSynchronize or an event). A caller that alternates
+ * two workspaces and two streams overlaps one step's copies with the other
+ * step's kernels; each step still copies its own input in and its output out.
+ */
+MOE_API int moe_forward_host_async(const moe_config* cfg, int64_t T, const void* x_host, const moe_weights* w,
+                                   void* out_host, void* workspace, size_t workspace_bytes, moe_stream_t stream);
 
 /* ---- stage entry points (each a part of moe_forward, for tests and tools) ---- */
 
@@ -168,7 +197,8 @@ MOE_API int moe_permute(const moe_config* cfg, int64_t T, const int32_t* topk_id
  * MOE_ERR_UNSUPPORTED_SHAPE without touching the device.
  * device_status (optional, device memory, one int) receives the device status
  * (MOE_ERR_BAD_INDEX for skipped pairs); the call zeroes it first. Without it
- * the status word lives in the shared scratch.
+ * the status word lives in the shared scratch, where no entry point can read
+ * it: a caller that needs to detect bad indices must pass device_status.
  * The first call with a given device current looks up the scratch address on
  * that device; make that first call before any stream capture. Every call
  * shares the one scratch array per device: calls whose work overlaps on the
@@ -187,10 +217,65 @@ MOE_API int moe_experts(const moe_config* cfg, int64_t T, const void* x, const i
                 const float* topk_w, const moe_weights* w, void* y, int32_t* pos, void* workspace,
                 size_t workspace_bytes, moe_stream_t stream);
 
+/* One grouped expert GEMM over rows already grouped by expert (the GEMMs of
+ * moe_experts, for tests and tools). Rows [offsets[g], offsets[g+1]) of A belong
+ * to group g (routed experts 0..E-1, then the shared expert when n_shared == 1);
+ * offsets [E+S+1] int32 (device) must start at 0, never decrease and end at most
+ * at R (otherwise MOE_ERR_INVALID_ARG is latched in the workspace status and
+ * nothing is computed). Rows past offsets[E+S] are not written.
+ *   stage MOE_STAGE_GATE_UP:     A [R, H]; out = h [R, I] = silu(A W1_g^T) * (A W3_g^T),
+ *                                bf16 (BF16 storage) or E4M3 codes with out_scale
+ *                                [R, I/128] fp32 (FP8: 1x128 blocks, scale = blockmax/448)
+ *   stage MOE_STAGE_GATE_UP_RAW: A [R, H]; out = fp32 [R, 2, I]: the gate sums
+ *                                A W1_g^T, then the up sums A W3_g^T (no SwiGLU)
+ *   stage MOE_STAGE_DOWN:        A [R, I]; out = y [R, H] bf16 = row_gate[r] * (A W2_g^T)
+ *                                (row_gate [R] fp32, device; NULL means 1)
+ * A is bf16 (BF16 storage) or E4M3 codes with a_scale [R, K/128] fp32 (FP8, K
+ * the reduction length). The workspace is moe_workspace_bytes for
+ * ceil(R / (top_k + n_shared)) tokens. Device status: moe_read_status. */
+enum { MOE_STAGE_GATE_UP = 1, MOE_STAGE_GATE_UP_RAW = 2, MOE_STAGE_DOWN = 3 };
+MOE_API int moe_grouped_gemm(const moe_config* cfg, int stage, int64_t R, const int32_t* offsets, const void* a,
+                             const float* a_scale, const moe_weights* w, const float* row_gate, void* out,
+                             float* out_scale, void* workspace, size_t workspace_bytes, moe_stream_t stream);
+
 /* Combine: out[t] = sum over slots j < k+S of y[pos[t, j]], fp32 in slot
  * order, rounded once to bf16. y [(k+S)T, H] bf16, pos [T, k+S], out [T, H]. */
 MOE_API int moe_combine(const moe_config* cfg, int64_t T, const void* y, const int32_t* pos, void* out,
                 moe_stream_t stream);
+
+/* ---- expert parallelism (StepFun "Step-5 minimal inference" README: the
+ * deployment at TP = EP = 8 places 44 of the 352 routed experts on each GPU,
+ * tokens replicated over the group; "Long-output stability": the ranks'
+ * partial results are added in rank order with FP32 accumulation) ---- */
+
+/* One rank's share of the layer. cfg->n_experts is the number of routed
+ * experts the router chooses from (all ranks'); this rank computes its routed
+ * experts [e0, e1) and, when cfg->n_shared == 1, the shared expert for tokens
+ * [shared_t0, shared_t1) (the shared expert is replicated on every rank and
+ * its rows divided by token). Every token is routed over all experts:
+ *   w->router_w [E, H], w->router_bias [E] or NULL: all experts;
+ *   w->w1, w->w3 [e1-e0, I, H], w->w2 [e1-e0, H, I] (+ FP8 scales): this
+ *     rank's experts only, expert e0 first; shared-expert weights: whole.
+ * partial [T, H] fp32 (device, written): for each token, the sum in slot order
+ * of the gate-weighted rows this rank computed (zero where it computed none),
+ * not rounded to bf16. Summing the ranks' partials over a partition of the
+ * experts and of the shared expert's tokens gives the layer output
+ * (moe_ep_reduce). topk_idx / topk_w as for moe_forward. The workspace is
+ * moe_workspace_bytes(cfg, T) (the whole layer's). Requires 0 <= e0 < e1 <= E. */
+MOE_API int moe_forward_ep_partial(const moe_config* cfg, int64_t T, const void* x, const moe_weights* w,
+                                   int32_t e0, int32_t e1, int64_t shared_t0, int64_t shared_t1, float* partial,
+                                   int32_t* topk_idx, float* topk_w, void* workspace, size_t workspace_bytes,
+                                   moe_stream_t stream);
+
+/* The ranks' partial outputs added in rank order: for t in [t0, t1),
+ * out[t] = bf16(partials[0][t] + partials[1][t] + ... + partials[n-1][t]),
+ * summed in fp32 in that order and rounded once (nearest even).
+ * partials: a host array of n_ranks (1..16) device pointers to [T, H] fp32
+ * buffers that this device can read (its own memory, or peers' memory mapped
+ * for peer access); out [T, H] bf16 (device; rows outside [t0, t1) untouched).
+ * All pointers 16-byte aligned; H a multiple of 128. */
+MOE_API int moe_ep_reduce(int32_t n_ranks, const float* const* partials, int64_t T, int32_t hidden, int64_t t0,
+                          int64_t t1, void* out, moe_stream_t stream);
 
 /* ---- the fp32 residual stream around the layer ----
  * (NeMo "Step-5-Preview" page, "Full-Depth H100 Benchmark" table: FP32 norms and
@@ -219,6 +304,23 @@ MOE_API int moe_combine_residual(const moe_config* cfg, int64_t T, const void* y
  * moe_route, moe_permute and moe_experts call clears it first). */
 MOE_API int moe_read_status(const void* workspace, moe_stream_t stream, int* device_status);
 
+/* Synchronises `stream`, then copies the workspace's status record:
+ * detail[0] = status word (as moe_read_status); for MOE_ERR_DEVICE_TIMEOUT,
+ * detail[1] = the wait site of the first timeout (kernel variant and wait:
+ * nonzero), detail[2] = its block index, detail[3] = that wait's progress
+ * counter. */
+MOE_API int moe_read_status_detail(const void* workspace, moe_stream_t stream, int* detail /* [4] */);
+
+/* Test hook of the bounded waits (process-wide; not for production use).
+ * MOE_INJECT_GEMM_NO_LOADS makes the expert GEMMs' producer issue no loads, so
+ * their consumers' first waits run out after wait_limit_ns and the call latches
+ * MOE_ERR_DEVICE_TIMEOUT with nothing in flight: every kernel still returns and
+ * the device stays usable. wait_limit_ns bounds every wait of the expert GEMMs
+ * (0 restores the default of 2 s). MOE_INJECT_NONE with 0 restores normal
+ * operation. */
+enum { MOE_INJECT_NONE = 0, MOE_INJECT_GEMM_NO_LOADS = 1 };
+MOE_API int moe_debug_inject(int what, uint64_t wait_limit_ns);
+
 /* Text for a status code (static storage). */
 MOE_API const char* moe_status_string(int status);
 
@@ -240,6 +342,10 @@ MOE_API const char* moe_profile_kernel_name(int i);
  * held to the same tolerance by the tests. */
 enum { MOE_GEMM_AUTO = 0, MOE_GEMM_SINGLE = 1, MOE_GEMM_PAIR = 2 };
 MOE_API int moe_set_gemm_variant(int variant);
+
+/* Kernels this library has launched in this process so far (every entry
+ * point, every device); the difference across a region counts its launches. */
+MOE_API int moe_launch_count(uint64_t* n);
 
 /* Number of streaming multiprocessors the kernels size their grids for
  * (current device). */

@@ -6,10 +6,12 @@ streams. The binding fails loudly when the library is missing or when a call
 returns an error; there is no fallback.
 
 The functions carry the names of the C entry points:
-  moe_workspace_bytes, moe_forward, moe_forward_host, moe_route,
+  moe_workspace_bytes, moe_forward, moe_forward_host, moe_forward_host_async, moe_route,
   moe_quantize_act, moe_permute, moe_experts, moe_combine, moe_read_status,
   moe_status_string, moe_profile_enable, moe_profile_read, moe_device_sm_count,
-  moe_set_gemm_variant, moe_permute_noalloc, moe_rmsnorm, moe_combine_residual.
+  moe_set_gemm_variant, moe_permute_noalloc, moe_rmsnorm, moe_combine_residual,
+  moe_grouped_gemm, moe_read_status_detail, moe_debug_inject, moe_launch_count,
+  moe_forward_ep_partial, moe_ep_reduce.
 """
 from __future__ import annotations
 
@@ -20,7 +22,7 @@ from typing import Optional
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "_lib", "libmoe_b200.so")
 
-MOE_WDTYPE_BF16, MOE_WDTYPE_FP8_E4M3 = 0, 1
+MOE_WDTYPE_BF16, MOE_WDTYPE_FP8_E4M3, MOE_WDTYPE_NVFP4 = 0, 1, 2
 MOE_OK = 0
 MOE_ERR_INVALID_ARG = 1
 MOE_ERR_UNSUPPORTED_SHAPE = 2
@@ -30,6 +32,8 @@ MOE_ERR_BAD_INDEX = 5
 MOE_ERR_DEVICE_TIMEOUT = 6
 MOE_ERR_MISALIGNED = 7
 MOE_GEMM_AUTO, MOE_GEMM_SINGLE, MOE_GEMM_PAIR = 0, 1, 2
+MOE_STAGE_GATE_UP, MOE_STAGE_GATE_UP_RAW, MOE_STAGE_DOWN = 1, 2, 3
+MOE_INJECT_NONE, MOE_INJECT_GEMM_NO_LOADS = 0, 1
 
 _lib = None
 
@@ -46,7 +50,7 @@ class moe_config(ctypes.Structure):
 
 
 WEIGHT_FIELDS = ("router_w", "router_bias", "w1", "w3", "w2", "s1", "s3", "s2",
-                 "sw1", "sw3", "sw2", "ss1", "ss3", "ss2")
+                 "sw1", "sw3", "sw2", "ss1", "ss3", "ss2", "g1", "g3", "g2", "sg1", "sg3", "sg2")
 
 
 class moe_weights(ctypes.Structure):
@@ -67,6 +71,7 @@ def load():
         "moe_workspace_bytes": [cfgp, i64, ctypes.POINTER(sz)],
         "moe_forward": [cfgp, i64, vp, wp, vp, vp, vp, vp, sz, vp],
         "moe_forward_host": [cfgp, i64, vp, wp, vp, vp, sz, vp],
+        "moe_forward_host_async": [cfgp, i64, vp, wp, vp, vp, sz, vp],
         "moe_route": [cfgp, i64, vp, vp, vp, vp, vp, vp, vp, sz, vp],
         "moe_quantize_act": [i64, i32, vp, vp, vp, vp],
         "moe_permute": [cfgp, i64, vp, vp, vp, vp, vp, vp, sz, vp],
@@ -82,6 +87,12 @@ def load():
         "moe_permute_noalloc": [cfgp, i64, vp, vp, vp, vp, vp, vp, vp],
         "moe_rmsnorm": [i64, i32, vp, vp, ctypes.c_float, vp, vp],
         "moe_combine_residual": [cfgp, i64, vp, vp, vp, vp, vp],
+        "moe_grouped_gemm": [cfgp, ctypes.c_int, i64, vp, vp, vp, wp, vp, vp, vp, vp, sz, vp],
+        "moe_read_status_detail": [vp, vp, ctypes.POINTER(ctypes.c_int)],
+        "moe_debug_inject": [ctypes.c_int, ctypes.c_uint64],
+        "moe_launch_count": [ctypes.POINTER(ctypes.c_uint64)],
+        "moe_forward_ep_partial": [cfgp, i64, vp, wp, i32, i32, i64, i64, vp, vp, vp, vp, sz, vp],
+        "moe_ep_reduce": [i32, ctypes.POINTER(ctypes.c_void_p), i64, i32, i64, i64, vp, vp],
     }
     for name, args in sig.items():
         f = getattr(lib, name)
@@ -148,6 +159,13 @@ def moe_forward_host(cfg, T, x_host, w: moe_weights, out_host, workspace, stream
                                    _ptr(workspace), nb, _stream(stream)), "moe_forward_host")
 
 
+def moe_forward_host_async(cfg, T, x_host, w: moe_weights, out_host, workspace, stream=None):
+    """moe_forward_host queued on `stream` without the final synchronisation."""
+    nb = workspace.numel() * workspace.element_size()
+    _check(load().moe_forward_host_async(ctypes.byref(cfg), T, _ptr(x_host), ctypes.byref(w), _ptr(out_host),
+                                         _ptr(workspace), nb, _stream(stream)), "moe_forward_host_async")
+
+
 def moe_route(cfg, T, x, router_w, router_bias, topk_idx, topk_w, logits, workspace, stream=None):
     nb = workspace.numel() * workspace.element_size()
     _check(load().moe_route(ctypes.byref(cfg), T, _ptr(x), _ptr(router_w), _ptr(router_bias), _ptr(topk_idx),
@@ -177,6 +195,32 @@ def moe_experts(cfg, T, x, topk_idx, topk_w, w: moe_weights, y, pos, workspace, 
                               _ptr(y), _ptr(pos), _ptr(workspace), nb, _stream(stream)), "moe_experts")
 
 
+def moe_forward_ep_partial(cfg, T, x, w: moe_weights, e0, e1, shared_t0, shared_t1, partial, workspace,
+                           topk_idx=None, topk_w=None, stream=None):
+    """One expert-parallel rank's fp32 partial output (its experts [e0, e1) and
+    its shared-expert tokens [shared_t0, shared_t1))."""
+    nb = workspace.numel() * workspace.element_size()
+    _check(load().moe_forward_ep_partial(ctypes.byref(cfg), T, _ptr(x), ctypes.byref(w), e0, e1, shared_t0,
+                                         shared_t1, _ptr(partial), _ptr(topk_idx), _ptr(topk_w), _ptr(workspace),
+                                         nb, _stream(stream)), "moe_forward_ep_partial")
+
+
+def moe_ep_reduce(partials, T, hidden, t0, t1, out, stream=None):
+    """out[t0:t1] = bf16 of the fp32 partials added in rank order."""
+    arr = (ctypes.c_void_p * len(partials))(*[_ptr(p) for p in partials])
+    _check(load().moe_ep_reduce(len(partials), arr, T, hidden, t0, t1, _ptr(out), _stream(stream)),
+           "moe_ep_reduce")
+
+
+def moe_grouped_gemm(cfg, stage, R, offsets, a, a_scale, w: moe_weights, out, workspace, row_gate=None,
+                     out_scale=None, stream=None):
+    """One grouped expert GEMM over rows grouped by `offsets` (MOE_STAGE_*)."""
+    nb = workspace.numel() * workspace.element_size()
+    _check(load().moe_grouped_gemm(ctypes.byref(cfg), stage, R, _ptr(offsets), _ptr(a), _ptr(a_scale),
+                                   ctypes.byref(w), _ptr(row_gate), _ptr(out), _ptr(out_scale), _ptr(workspace),
+                                   nb, _stream(stream)), "moe_grouped_gemm")
+
+
 def moe_combine(cfg, T, y, pos, out, stream=None):
     _check(load().moe_combine(ctypes.byref(cfg), T, _ptr(y), _ptr(pos), _ptr(out), _stream(stream)),
            "moe_combine")
@@ -200,6 +244,18 @@ def moe_read_status(workspace, stream=None) -> int:
     return v.value
 
 
+def moe_read_status_detail(workspace, stream=None):
+    """(status, wait site, block, progress) of the workspace's status record."""
+    v = (ctypes.c_int * 4)()
+    _check(load().moe_read_status_detail(_ptr(workspace), _stream(stream), v), "moe_read_status_detail")
+    return tuple(int(x) for x in v)
+
+
+def moe_debug_inject(what: int, wait_limit_ns: int = 0):
+    """Test hook of the expert GEMMs' bounded waits (MOE_INJECT_*)."""
+    _check(load().moe_debug_inject(what, wait_limit_ns), "moe_debug_inject")
+
+
 def moe_profile_enable(on: bool):
     _check(load().moe_profile_enable(1 if on else 0), "moe_profile_enable")
 
@@ -215,6 +271,13 @@ def moe_profile_read() -> dict:
 
 def moe_set_gemm_variant(variant: int):
     _check(load().moe_set_gemm_variant(variant), "moe_set_gemm_variant")
+
+
+def moe_launch_count() -> int:
+    """Kernels the library has launched in this process so far."""
+    v = ctypes.c_uint64(0)
+    _check(load().moe_launch_count(ctypes.byref(v)), "moe_launch_count")
+    return v.value
 
 
 def moe_device_sm_count() -> int:

@@ -4,10 +4,12 @@
 #include <stdio.h>
 #include <string.h>
 
+#include <atomic>
 #include <mutex>
 
 #include "common.cuh"
 #include "moe.h"
+#include "ptx.cuh"
 
 namespace moe {
 
@@ -54,6 +56,20 @@ bool map_2d(CUtensorMap* m, const void* base, bool fp8, uint64_t inner, uint64_t
   return r == CUDA_SUCCESS;
 }
 
+// 2-D uint8 tensor map without swizzle (NVFP4 codes and scales): rows of
+// `inner` bytes, boxes of box_inner bytes x box_outer rows.
+bool map_u8(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint32_t box_inner,
+            uint32_t box_outer) {
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {inner};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t estr[2] = {1, 1};
+  const CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+                              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
 
 int check_config(const moe_config* c, int64_t T) {
@@ -61,8 +77,11 @@ int check_config(const moe_config* c, int64_t T) {
   if (T < 0) return MOE_ERR_INVALID_ARG;
   if (c->hidden <= 0 || c->inter <= 0 || c->n_experts <= 0 || c->top_k <= 0) return MOE_ERR_INVALID_ARG;
   if (c->n_shared < 0 || c->n_shared > 1) return MOE_ERR_UNSUPPORTED_SHAPE;
-  if (c->wdtype != MOE_WDTYPE_BF16 && c->wdtype != MOE_WDTYPE_FP8_E4M3) return MOE_ERR_INVALID_ARG;
+  if (c->wdtype != MOE_WDTYPE_BF16 && c->wdtype != MOE_WDTYPE_FP8_E4M3 && c->wdtype != MOE_WDTYPE_NVFP4)
+    return MOE_ERR_INVALID_ARG;
   if (c->hidden % 128 || c->inter % 128) return MOE_ERR_UNSUPPORTED_SHAPE;
+  // NVFP4: the scale tensors' rows (K/16 bytes) must be whole 16-byte TMA strides.
+  if (c->wdtype == MOE_WDTYPE_NVFP4 && (c->hidden % 256 || c->inter % 256)) return MOE_ERR_UNSUPPORTED_SHAPE;
   if (c->n_experts > kMaxExperts || c->top_k > kMaxTopK || c->top_k > c->n_experts) return MOE_ERR_UNSUPPORTED_SHAPE;
   if ((int64_t)(c->top_k + c->n_shared) * T >= ((int64_t)1 << 31) - 256) return MOE_ERR_UNSUPPORTED_SHAPE;
   if ((int64_t)c->n_experts * c->hidden >= ((int64_t)1 << 31) || (int64_t)c->n_experts * c->inter >= ((int64_t)1 << 31))
@@ -73,19 +92,24 @@ int check_config(const moe_config* c, int64_t T) {
 int check_weights(const moe_config* c, const moe_weights* w) {
   if (!w) return MOE_ERR_INVALID_ARG;
   const bool fp8 = c->wdtype == MOE_WDTYPE_FP8_E4M3;
+  const bool nv = c->wdtype == MOE_WDTYPE_NVFP4;
   const void* need[] = {w->router_w, w->w1, w->w3, w->w2};
   for (const void* p : need) {
     if (!p) return MOE_ERR_INVALID_ARG;
     if (!aligned(p, 16)) return MOE_ERR_MISALIGNED;
   }
-  if (fp8 && (!w->s1 || !w->s3 || !w->s2)) return MOE_ERR_INVALID_ARG;
+  if ((fp8 || nv) && (!w->s1 || !w->s3 || !w->s2)) return MOE_ERR_INVALID_ARG;
+  if (nv && (!w->g1 || !w->g3 || !w->g2)) return MOE_ERR_INVALID_ARG;
+  if (nv && (!aligned(w->s1, 16) || !aligned(w->s3, 16) || !aligned(w->s2, 16))) return MOE_ERR_MISALIGNED;
   if (c->n_shared) {
     const void* sh[] = {w->sw1, w->sw3, w->sw2};
     for (const void* p : sh) {
       if (!p) return MOE_ERR_INVALID_ARG;
       if (!aligned(p, 16)) return MOE_ERR_MISALIGNED;
     }
-    if (fp8 && (!w->ss1 || !w->ss3 || !w->ss2)) return MOE_ERR_INVALID_ARG;
+    if ((fp8 || nv) && (!w->ss1 || !w->ss3 || !w->ss2)) return MOE_ERR_INVALID_ARG;
+    if (nv && (!w->sg1 || !w->sg3 || !w->sg2)) return MOE_ERR_INVALID_ARG;
+    if (nv && (!aligned(w->ss1, 16) || !aligned(w->ss3, 16) || !aligned(w->ss2, 16))) return MOE_ERR_MISALIGNED;
   }
   return MOE_OK;
 }
@@ -124,11 +148,6 @@ struct Prof {
   ~Prof() {
     if (on) g_prof_recorded = n;
   }
-};
-
-struct Maps {
-  CUtensorMap x, wr, w1, w3, sw1, sw3, w2, sw2, w2h, sw2h;  // w2h/sw2h: 128-row boxes
-  AMaps xp, h;                                           // GEMM1 / GEMM2 activations
 };
 
 void router_shape(int E, int* nbox, int* box_rows) {
@@ -190,6 +209,10 @@ PermuteParams permute_params(const moe_config* c, const WsLayout& L, int64_t T, 
   pp.k = c->top_k;
   pp.S = c->n_shared;
   pp.G = c->n_experts + c->n_shared;
+  pp.e0 = 0;
+  pp.E_all = c->n_experts;
+  pp.sh_t0 = 0;
+  pp.sh_t1 = (int32_t)T;
   pp.chunks = (int32_t)L.chunks;
   pp.idx = idx;
   pp.gate = gate;
@@ -224,23 +247,212 @@ int run_permute(const PermuteParams& pp, cudaStream_t s, Prof& prof) {
   return MOE_OK;
 }
 
-// gather + GEMM1 + GEMM2 for a permutation already in the workspace; y [R, H] bf16.
-int run_experts(const moe_config* c, const WsLayout& L, int64_t T, const void* x, const moe_weights* w,
-                const int32_t* pos, void* y, uint8_t* ws, cudaStream_t s, Prof& prof) {
+// Process-wide test hooks of the expert GEMMs (moe_debug_inject).
+uint64_t g_wait_ns = kWaitLimitNs;
+int g_inject = 0;
+
+// GEMM1 runs on 2-SM pairs under AUTO when the routed groups average at least
+// kPairMinRows rows.
+bool gate_up_on_pairs(int64_t routed_rows, int n_experts) {
+  return g_gemm_variant == MOE_GEMM_PAIR ||
+         (g_gemm_variant == MOE_GEMM_AUTO && routed_rows >= kPairMinRows * (int64_t)n_experts);
+}
+
+bool amaps(AMaps* a, const void* base, bool fp8, uint64_t inner, uint64_t rows) {
+  const uint32_t box_k = fp8 ? 128 : 64;
+  return map_2d(&a->rows128, base, fp8, inner, rows, box_k, 128) &&
+         map_2d(&a->rows64, base, fp8, inner, rows, box_k, 64) && map_2d(&a->rows32, base, fp8, inner, rows, box_k, 32);
+}
+
+// The grouped gate/up GEMM (GEMM1) over R rows of A [R, H] grouped by `offsets`
+// (tile prefixes mt / mp for single CTAs / pairs). FP8: a_scale_t [H/128,
+// rows_pad]; out = h codes [R, I] with out_scale_t [I/128, rows_pad]. BF16: out
+// = h [R, I] bf16. raw: out = fp32 [R, 2I] gate and up sums (no SwiGLU).
+int run_gate_up(const moe_config* c, const WsLayout& L, int64_t R, const void* a, const float* a_scale_t,
+                const int32_t* offsets, const int32_t* mt, const int32_t* mp, bool pair, const moe_weights* w,
+                void* out, float* out_scale_t, bool raw, int* status, cudaStream_t s) {
   if (!get_encoder()) return MOE_ERR_CUDA;
   const bool fp8 = c->wdtype == MOE_WDTYPE_FP8_E4M3;
   const int H = c->hidden, I = c->inter, E = c->n_experts, S = c->n_shared;
-  const int es = fp8 ? 1 : 2;
-  const uint32_t box_k = 128 / es;
-  const int64_t R = L.R;
+  const uint32_t box_k = fp8 ? 128 : 64;
   const int sms = sm_count();
   if (sms <= 0) return MOE_ERR_CUDA;
-  const bool pair = g_gemm_variant == MOE_GEMM_PAIR;  // GEMM2 (and the maps it shares)
-  const bool pair1 = pair || (g_gemm_variant == MOE_GEMM_AUTO && (int64_t)c->top_k * T >= kPairMinRows * E);
+  AMaps ma;
+  if (c->wdtype == MOE_WDTYPE_NVFP4) {
+    // W4A16: bf16 activations; codes [E I, H/2] and scales [E I, H/16] per matrix.
+    NvMaps nm;
+    bool ok = amaps(&ma, a, false, H, R) && map_u8(&nm.code0, w->w1, H / 2, (uint64_t)E * I, 32, 128) &&
+              map_u8(&nm.code1, w->w3, H / 2, (uint64_t)E * I, 32, 128) &&
+              map_u8(&nm.scale0, w->s1, H / 16, (uint64_t)E * I, 16, 128) &&
+              map_u8(&nm.scale1, w->s3, H / 16, (uint64_t)E * I, 16, 128);
+    if (S) {
+      ok = ok && map_u8(&nm.scode0, w->sw1, H / 2, I, 32, 128) && map_u8(&nm.scode1, w->sw3, H / 2, I, 32, 128) &&
+           map_u8(&nm.sscale0, w->ss1, H / 16, I, 16, 128) && map_u8(&nm.sscale1, w->ss3, H / 16, I, 16, 128);
+    } else {
+      nm.scode0 = nm.code0;
+      nm.scode1 = nm.code1;
+      nm.sscale0 = nm.scale0;
+      nm.sscale1 = nm.scale1;
+    }
+    if (!ok) return MOE_ERR_CUDA;
+    GemmParams g{};
+    g.mt_prefix = mt;
+    g.offsets = offsets;
+    g.G = E + S;
+    g.E = E;
+    g.K = H;
+    g.N = I;
+    g.n_tiles = I / 128;
+    g.n_fastest = 0;
+    g.R = (int32_t)R;
+    g.rows_pad = L.rows_pad;
+    g.b_scale0 = w->g1;
+    g.b_scale1 = w->g3;
+    g.bs_scale0 = w->sg1;
+    g.bs_scale1 = w->sg3;
+    g.out = out;
+    g.status = status;
+    g.wait_ns = g_wait_ns;
+    g.raw_out = raw ? 1 : 0;
+    g.inject = g_inject;
+    CUDA_TRY(launch_nvfp4_gemm(g, true, sms, ma, nm, s));
+    return MOE_OK;
+  }
+  CUtensorMap w1, w3, sw1, sw3;
+  bool ok = amaps(&ma, a, fp8, H, R) && map_2d(&w1, w->w1, fp8, H, (uint64_t)E * I, box_k, 128) &&
+            map_2d(&w3, w->w3, fp8, H, (uint64_t)E * I, box_k, 128);
+  if (S) {
+    ok = ok && map_2d(&sw1, w->sw1, fp8, H, I, box_k, 128) && map_2d(&sw3, w->sw3, fp8, H, I, box_k, 128);
+  } else {
+    sw1 = w1;
+    sw3 = w3;
+  }
+  if (!ok) return MOE_ERR_CUDA;
+  GemmParams g{};
+  g.mt_prefix = pair ? mp : mt;
+  g.offsets = offsets;
+  g.G = E + S;
+  g.E = E;
+  g.K = H;
+  g.N = I;
+  g.n_tiles = I / 128;
+  g.n_fastest = 0;
+  g.R = (int32_t)R;
+  g.rows_pad = L.rows_pad;
+  g.a_scale = fp8 ? a_scale_t : nullptr;
+  g.b_scale0 = w->s1;
+  g.b_scale1 = w->s3;
+  g.bs_scale0 = w->ss1;
+  g.bs_scale1 = w->ss3;
+  g.out = out;
+  g.out_scale = fp8 ? out_scale_t : nullptr;
+  g.row_gate = nullptr;
+  g.status = status;
+  g.wait_ns = g_wait_ns;
+  g.raw_out = raw ? 1 : 0;
+  g.inject = g_inject;
+  CUDA_TRY(launch_gemm1(g, fp8, pair, sms, ma, w1, w3, sw1, sw3, s));
+  return MOE_OK;
+}
 
+// The grouped down GEMM (GEMM2): y [R, H] bf16 = row_gate[r] * (A W2_g^T) for
+// A [R, I] (FP8: codes with a_scale_t [I/128, rows_pad]); row_gate may be null (1).
+int run_down(const moe_config* c, const WsLayout& L, int64_t R, const void* a, const float* a_scale_t,
+             const int32_t* offsets, const int32_t* mt, const int32_t* mp, bool pair, const moe_weights* w,
+             const float* row_gate, void* y, int* status, cudaStream_t s) {
+  if (!get_encoder()) return MOE_ERR_CUDA;
+  const bool fp8 = c->wdtype == MOE_WDTYPE_FP8_E4M3;
+  const int H = c->hidden, I = c->inter, E = c->n_experts, S = c->n_shared;
+  const uint32_t box_k = fp8 ? 128 : 64;
+  const int sms = sm_count();
+  if (sms <= 0) return MOE_ERR_CUDA;
+  AMaps ma;
+  if (c->wdtype == MOE_WDTYPE_NVFP4) {
+    NvMaps nm;
+    bool ok = amaps(&ma, a, false, I, R) && map_u8(&nm.code0, w->w2, I / 2, (uint64_t)E * H, 32, 256) &&
+              map_u8(&nm.scale0, w->s2, I / 16, (uint64_t)E * H, 16, 256);
+    if (S) {
+      ok = ok && map_u8(&nm.scode0, w->sw2, I / 2, H, 32, 256) && map_u8(&nm.sscale0, w->ss2, I / 16, H, 16, 256);
+    } else {
+      nm.scode0 = nm.code0;
+      nm.sscale0 = nm.scale0;
+    }
+    nm.code1 = nm.code0;
+    nm.scode1 = nm.scode0;
+    nm.scale1 = nm.scale0;
+    nm.sscale1 = nm.sscale0;
+    if (!ok) return MOE_ERR_CUDA;
+    GemmParams g{};
+    g.mt_prefix = mt;
+    g.offsets = offsets;
+    g.G = E + S;
+    g.E = E;
+    g.K = I;
+    g.N = H;
+    g.n_tiles = (int32_t)ceil_div(H, 256);
+    g.n_fastest = 1;
+    g.R = (int32_t)R;
+    g.rows_pad = L.rows_pad;
+    g.b_scale0 = w->g2;
+    g.b_scale1 = w->g2;
+    g.bs_scale0 = w->sg2;
+    g.bs_scale1 = w->sg2;
+    g.out = y;
+    g.row_gate = row_gate;
+    g.status = status;
+    g.wait_ns = g_wait_ns;
+    g.inject = g_inject;
+    CUDA_TRY(launch_nvfp4_gemm(g, false, sms, ma, nm, s));
+    return MOE_OK;
+  }
+  CUtensorMap w2, w2h, sw2, sw2h;
+  bool ok = amaps(&ma, a, fp8, I, R) && map_2d(&w2, w->w2, fp8, I, (uint64_t)E * H, box_k, 256) &&
+            map_2d(&w2h, w->w2, fp8, I, (uint64_t)E * H, box_k, 128);
+  if (S) {
+    ok = ok && map_2d(&sw2, w->sw2, fp8, I, H, box_k, 256) && map_2d(&sw2h, w->sw2, fp8, I, H, box_k, 128);
+  } else {
+    sw2 = w2;
+    sw2h = w2h;
+  }
+  if (!ok) return MOE_ERR_CUDA;
+  GemmParams g{};
+  g.mt_prefix = pair ? mp : mt;
+  g.offsets = offsets;
+  g.G = E + S;
+  g.E = E;
+  g.K = I;
+  g.N = H;
+  g.n_tiles = (int32_t)ceil_div(H, 256);
+  g.n_fastest = 1;
+  g.R = (int32_t)R;
+  g.rows_pad = L.rows_pad;
+  g.a_scale = fp8 ? a_scale_t : nullptr;
+  g.b_scale0 = w->s2;
+  g.b_scale1 = w->s2;
+  g.bs_scale0 = w->ss2;
+  g.bs_scale1 = w->ss2;
+  g.out = y;
+  g.out_scale = nullptr;
+  g.row_gate = row_gate;
+  g.status = status;
+  g.wait_ns = g_wait_ns;
+  g.raw_out = 0;
+  g.inject = g_inject;
+  CUDA_TRY(launch_gemm2(g, fp8, pair, sms, ma, w2, w2h, sw2, sw2h, s));
+  return MOE_OK;
+}
+
+// gather + GEMM1 + GEMM2 for a permutation already in the workspace; y [R, H] bf16.
+// routed_rows: the routed rows this call expects (k T on one GPU), which
+// decides whether the gate/up GEMM runs on 2-SM pairs.
+int run_experts(const moe_config* c, const WsLayout& L, int64_t T, const void* x, const moe_weights* w,
+                const int32_t* pos, void* y, uint8_t* ws, cudaStream_t s, Prof& prof, int64_t routed_rows) {
+  const bool fp8 = c->wdtype == MOE_WDTYPE_FP8_E4M3;
+  const int S = c->n_shared;
+  const int64_t R = L.R;
   GatherParams gp{};
   gp.T = (int32_t)T;
-  gp.H = H;
+  gp.H = c->hidden;
   gp.S = c->top_k + S;
   gp.rows_pad = L.rows_pad;
   gp.x = static_cast<const uint16_t*>(x);
@@ -251,65 +463,19 @@ int run_experts(const moe_config* c, const WsLayout& L, int64_t T, const void* x
   CUDA_TRY(launch_gather(gp, fp8, s));
   prof.mark();
 
-  Maps m;
-  auto amaps = [&](AMaps* a, const void* base, uint64_t inner) {
-    return map_2d(&a->rows128, base, fp8, inner, R, box_k, 128) && map_2d(&a->rows64, base, fp8, inner, R, box_k, 64) &&
-           map_2d(&a->rows32, base, fp8, inner, R, box_k, 32);
-  };
-  bool ok = amaps(&m.xp, ws + L.xp, H) && amaps(&m.h, ws + L.h, I) &&
-            map_2d(&m.w1, w->w1, fp8, H, (uint64_t)E * I, box_k, 128) &&
-            map_2d(&m.w3, w->w3, fp8, H, (uint64_t)E * I, box_k, 128) &&
-            map_2d(&m.w2, w->w2, fp8, I, (uint64_t)E * H, box_k, 256) &&
-            map_2d(&m.w2h, w->w2, fp8, I, (uint64_t)E * H, box_k, 128);
-  if (S) {
-    ok = ok && map_2d(&m.sw1, w->sw1, fp8, H, I, box_k, 128) && map_2d(&m.sw3, w->sw3, fp8, H, I, box_k, 128) &&
-         map_2d(&m.sw2, w->sw2, fp8, I, H, box_k, 256) && map_2d(&m.sw2h, w->sw2, fp8, I, H, box_k, 128);
-  } else {
-    m.sw1 = m.w1;
-    m.sw3 = m.w3;
-    m.sw2 = m.w2;
-    m.sw2h = m.w2h;
-  }
-  if (!ok) return MOE_ERR_CUDA;
-
-  GemmParams g1{};
-  g1.mt_prefix = reinterpret_cast<const int32_t*>(ws + (pair1 ? L.mp_prefix : L.mt_prefix));
-  g1.offsets = reinterpret_cast<const int32_t*>(ws + L.offsets);
-  g1.G = E + S;
-  g1.E = E;
-  g1.K = H;
-  g1.N = I;
-  g1.n_tiles = I / 128;
-  g1.n_fastest = 0;
-  g1.R = (int32_t)R;
-  g1.rows_pad = L.rows_pad;
-  g1.a_scale = fp8 ? reinterpret_cast<const float*>(ws + L.sxp) : nullptr;
-  g1.b_scale0 = w->s1;
-  g1.b_scale1 = w->s3;
-  g1.bs_scale0 = w->ss1;
-  g1.bs_scale1 = w->ss3;
-  g1.out = ws + L.h;
-  g1.out_scale = fp8 ? reinterpret_cast<float*>(ws + L.sh) : nullptr;
-  g1.row_gate = nullptr;
-  g1.status = reinterpret_cast<int*>(ws + L.status);
-  CUDA_TRY(launch_gemm1(g1, fp8, pair1, sms, m.xp, m.w1, m.w3, m.sw1, m.sw3, s));
+  const int32_t* offsets = reinterpret_cast<const int32_t*>(ws + L.offsets);
+  const int32_t* mt = reinterpret_cast<const int32_t*>(ws + L.mt_prefix);
+  const int32_t* mp = reinterpret_cast<const int32_t*>(ws + L.mp_prefix);
+  int* status = reinterpret_cast<int*>(ws + L.status);
+  const bool pair2 = g_gemm_variant == MOE_GEMM_PAIR;
+  const bool pair1 = gate_up_on_pairs(routed_rows, c->n_experts);
+  int rc = run_gate_up(c, L, R, ws + L.xp, reinterpret_cast<const float*>(ws + L.sxp), offsets, mt, mp, pair1, w,
+                       ws + L.h, reinterpret_cast<float*>(ws + L.sh), false, status, s);
+  if (rc != MOE_OK) return rc;
   prof.mark();
-
-  GemmParams g2 = g1;
-  g2.mt_prefix = reinterpret_cast<const int32_t*>(ws + (pair ? L.mp_prefix : L.mt_prefix));
-  g2.K = I;
-  g2.N = H;
-  g2.n_tiles = (int32_t)ceil_div(H, 256);
-  g2.n_fastest = 1;
-  g2.a_scale = fp8 ? reinterpret_cast<const float*>(ws + L.sh) : nullptr;
-  g2.b_scale0 = w->s2;
-  g2.b_scale1 = w->s2;
-  g2.bs_scale0 = w->ss2;
-  g2.bs_scale1 = w->ss2;
-  g2.out = y;
-  g2.out_scale = nullptr;
-  g2.row_gate = reinterpret_cast<const float*>(ws + L.row_gate);
-  CUDA_TRY(launch_gemm2(g2, fp8, pair, sms, m.h, m.w2, m.w2h, m.sw2, m.sw2h, s));
+  rc = run_down(c, L, R, ws + L.h, reinterpret_cast<const float*>(ws + L.sh), offsets, mt, mp, pair2, w,
+                reinterpret_cast<const float*>(ws + L.row_gate), y, status, s);
+  if (rc != MOE_OK) return rc;
   prof.mark();
   return MOE_OK;
 }
@@ -338,6 +504,13 @@ int check_ws(const moe_config* c, int64_t T, void* ws, size_t ws_bytes, WsLayout
 
 }  // namespace
 
+std::atomic<uint64_t> g_launches{0};
+
+cudaError_t counted_launch(cudaError_t e) {
+  if (e == cudaSuccess) g_launches.fetch_add(1, std::memory_order_relaxed);
+  return e;
+}
+
 WsLayout ws_layout(const moe_config& c, int64_t T, int target_ctas) {
   WsLayout L{};
   const int S = c.n_shared, k = c.top_k, E = c.n_experts, G = E + S;
@@ -357,7 +530,7 @@ WsLayout ws_layout(const moe_config& c, int64_t T, int target_ctas) {
     off = (size_t)round_up((int64_t)(off + (bytes ? bytes : 1)), 1024);
     return o;
   };
-  L.status = take(16384);  // status word, first-timeout record, debug counters
+  L.status = take(kStatusBytes);  // status word, first-timeout record, debug counters
   L.idx = take((size_t)T * k * 4);
   L.gate = take((size_t)T * k * 4);
   L.logits_part = take((size_t)L.ksplit * T * E * 4);
@@ -407,19 +580,19 @@ int moe_forward(const moe_config* cfg, int64_t T, const void* x, const moe_weigh
   if (T == 0) return MOE_OK;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
-  CUDA_TRY(cudaMemsetAsync(ws + L.status, 0, 16384, s));
+  CUDA_TRY(cudaMemsetAsync(ws + L.status, 0, kStatusBytes, s));
   Prof prof(s);
   int32_t* idx = topk_idx ? topk_idx : reinterpret_cast<int32_t*>(ws + L.idx);
   float* gate = topk_w ? topk_w : reinterpret_cast<float*>(ws + L.gate);
   if ((rc = run_route(cfg, L, T, x, w->router_w, w->router_bias, idx, gate, nullptr, ws, s, prof)) != MOE_OK) return rc;
   const PermuteParams pp = permute_params(cfg, L, T, idx, gate, ws);
   if ((rc = run_permute(pp, s, prof)) != MOE_OK) return rc;
-  if ((rc = run_experts(cfg, L, T, x, w, pp.pos, ws + L.y, ws, s, prof)) != MOE_OK) return rc;
+  if ((rc = run_experts(cfg, L, T, x, w, pp.pos, ws + L.y, ws, s, prof, (int64_t)cfg->top_k * T)) != MOE_OK) return rc;
   return run_combine(cfg, T, ws + L.y, pp.pos, out, s, prof);
 }
 
-int moe_forward_host(const moe_config* cfg, int64_t T, const void* x_host, const moe_weights* w, void* out_host,
-                     void* workspace, size_t workspace_bytes, moe_stream_t stream) {
+int moe_forward_host_async(const moe_config* cfg, int64_t T, const void* x_host, const moe_weights* w,
+                           void* out_host, void* workspace, size_t workspace_bytes, moe_stream_t stream) {
   int rc = check_config(cfg, T);
   if (rc != MOE_OK) return rc;
   if (!x_host || !out_host) return MOE_ERR_INVALID_ARG;
@@ -433,7 +606,51 @@ int moe_forward_host(const moe_config* cfg, int64_t T, const void* x_host, const
   rc = moe_forward(cfg, T, ws + L.x_stage, w, ws + L.out_stage, nullptr, nullptr, workspace, workspace_bytes, stream);
   if (rc != MOE_OK) return rc;
   CUDA_TRY(cudaMemcpyAsync(out_host, ws + L.out_stage, bytes, cudaMemcpyDeviceToHost, s));
-  CUDA_TRY(cudaStreamSynchronize(s));
+  return MOE_OK;
+}
+
+int moe_forward_host(const moe_config* cfg, int64_t T, const void* x_host, const moe_weights* w, void* out_host,
+                     void* workspace, size_t workspace_bytes, moe_stream_t stream) {
+  const int rc = moe_forward_host_async(cfg, T, x_host, w, out_host, workspace, workspace_bytes, stream);
+  if (rc != MOE_OK || T == 0) return rc;
+  CUDA_TRY(cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)));
+  return MOE_OK;
+}
+
+int moe_forward_ep_partial(const moe_config* cfg, int64_t T, const void* x, const moe_weights* w, int32_t e0,
+                           int32_t e1, int64_t shared_t0, int64_t shared_t1, float* partial, int32_t* topk_idx,
+                           float* topk_w, void* workspace, size_t workspace_bytes, moe_stream_t stream) {
+  int rc = check_config(cfg, T);
+  if (rc != MOE_OK) return rc;
+  if (e0 < 0 || e1 <= e0 || e1 > cfg->n_experts) return MOE_ERR_INVALID_ARG;
+  if (cfg->n_shared && (shared_t0 < 0 || shared_t1 < shared_t0 || shared_t1 > T)) return MOE_ERR_INVALID_ARG;
+  moe_config lc = *cfg;  // this rank's routed experts only
+  lc.n_experts = e1 - e0;
+  if ((rc = check_weights(&lc, w)) != MOE_OK) return rc;
+  if (!x || !partial) return MOE_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(partial, 16)) return MOE_ERR_MISALIGNED;
+  if ((topk_idx == nullptr) != (topk_w == nullptr)) return MOE_ERR_INVALID_ARG;
+  WsLayout L;
+  if ((rc = check_ws(cfg, T, workspace, workspace_bytes, &L)) != MOE_OK) return rc;
+  if (T == 0) return MOE_OK;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  CUDA_TRY(cudaMemsetAsync(ws + L.status, 0, kStatusBytes, s));
+  Prof prof(s);
+  prof.on = false;
+  int32_t* idx = topk_idx ? topk_idx : reinterpret_cast<int32_t*>(ws + L.idx);
+  float* gate = topk_w ? topk_w : reinterpret_cast<float*>(ws + L.gate);
+  if ((rc = run_route(cfg, L, T, x, w->router_w, w->router_bias, idx, gate, nullptr, ws, s, prof)) != MOE_OK) return rc;
+  PermuteParams pp = permute_params(&lc, L, T, idx, gate, ws);
+  pp.e0 = e0;
+  pp.E_all = cfg->n_experts;
+  pp.sh_t0 = cfg->n_shared ? (int32_t)shared_t0 : 0;
+  pp.sh_t1 = cfg->n_shared ? (int32_t)shared_t1 : 0;
+  if ((rc = run_permute(pp, s, prof)) != MOE_OK) return rc;
+  // The gate/up GEMM's variant follows the rows a routed group gets on average.
+  const int64_t routed_rows = (int64_t)cfg->top_k * T * lc.n_experts / cfg->n_experts;
+  if ((rc = run_experts(&lc, L, T, x, w, pp.pos, ws + L.y, ws, s, prof, routed_rows)) != MOE_OK) return rc;
+  CUDA_TRY(launch_ep_partial(T, cfg->hidden, cfg->top_k + cfg->n_shared, ws + L.y, pp.pos, partial, s));
   return MOE_OK;
 }
 
@@ -449,7 +666,7 @@ int moe_route(const moe_config* cfg, int64_t T, const void* x, const void* route
   if (T == 0) return MOE_OK;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
-  CUDA_TRY(cudaMemsetAsync(ws + L.status, 0, 16384, s));
+  CUDA_TRY(cudaMemsetAsync(ws + L.status, 0, kStatusBytes, s));
   Prof prof(s);
   prof.on = false;
   return run_route(cfg, L, T, x, router_w, router_bias, topk_idx, topk_w, logits, ws, s, prof);
@@ -483,7 +700,7 @@ int moe_permute(const moe_config* cfg, int64_t T, const int32_t* topk_idx, int32
   if ((rc = check_ws(cfg, T, workspace, workspace_bytes, &L)) != MOE_OK) return rc;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
-  CUDA_TRY(cudaMemsetAsync(ws + L.status, 0, 16384, s));
+  CUDA_TRY(cudaMemsetAsync(ws + L.status, 0, kStatusBytes, s));
   if (T == 0) {
     const int G = cfg->n_experts + cfg->n_shared;
     CUDA_TRY(cudaMemsetAsync(counts, 0, (size_t)G * 4, s));
@@ -513,13 +730,13 @@ int moe_experts(const moe_config* cfg, int64_t T, const void* x, const int32_t* 
   if (T == 0) return MOE_OK;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
-  CUDA_TRY(cudaMemsetAsync(ws + L.status, 0, 16384, s));
+  CUDA_TRY(cudaMemsetAsync(ws + L.status, 0, kStatusBytes, s));
   Prof prof(s);
   prof.on = false;
   PermuteParams pp = permute_params(cfg, L, T, topk_idx, topk_w, ws);
   pp.pos = pos;
   if ((rc = run_permute(pp, s, prof)) != MOE_OK) return rc;
-  return run_experts(cfg, L, T, x, w, pos, y, ws, s, prof);
+  return run_experts(cfg, L, T, x, w, pos, y, ws, s, prof, (int64_t)cfg->top_k * T);
 }
 
 int moe_combine(const moe_config* cfg, int64_t T, const void* y, const int32_t* pos, void* out, moe_stream_t stream) {
@@ -531,6 +748,67 @@ int moe_combine(const moe_config* cfg, int64_t T, const void* y, const int32_t* 
   Prof prof(reinterpret_cast<cudaStream_t>(stream));
   prof.on = false;
   return run_combine(cfg, T, y, pos, out, reinterpret_cast<cudaStream_t>(stream), prof);
+}
+
+int moe_grouped_gemm(const moe_config* cfg, int stage, int64_t R, const int32_t* offsets, const void* a,
+                     const float* a_scale, const moe_weights* w, const float* row_gate, void* out, float* out_scale,
+                     void* workspace, size_t workspace_bytes, moe_stream_t stream) {
+  int rc = check_config(cfg, 0);
+  if (rc != MOE_OK) return rc;
+  if ((rc = check_weights(cfg, w)) != MOE_OK) return rc;
+  if (stage != MOE_STAGE_GATE_UP && stage != MOE_STAGE_GATE_UP_RAW && stage != MOE_STAGE_DOWN)
+    return MOE_ERR_INVALID_ARG;
+  if (R < 0 || !offsets || !a || !out) return MOE_ERR_INVALID_ARG;
+  if (R >= ((int64_t)1 << 31) - 512) return MOE_ERR_UNSUPPORTED_SHAPE;
+  const bool fp8 = cfg->wdtype == MOE_WDTYPE_FP8_E4M3;
+  if (fp8 && !a_scale) return MOE_ERR_INVALID_ARG;
+  if (fp8 && stage == MOE_STAGE_GATE_UP && !out_scale) return MOE_ERR_INVALID_ARG;
+  if (!aligned(a, 16) || !aligned(out, 16) || !aligned(offsets, 4)) return MOE_ERR_MISALIGNED;
+  // The workspace of moe_forward for ceil(R / (top_k + n_shared)) tokens holds
+  // every scratch buffer this needs.
+  const int64_t T = ceil_div(R, cfg->top_k + cfg->n_shared);
+  if ((rc = check_config(cfg, T)) != MOE_OK) return rc;
+  WsLayout L;
+  if ((rc = check_ws(cfg, T, workspace, workspace_bytes, &L)) != MOE_OK) return rc;
+  if (R == 0) return MOE_OK;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  int* status = reinterpret_cast<int*>(ws + L.status);
+  CUDA_TRY(cudaMemsetAsync(ws + L.status, 0, kStatusBytes, s));
+  const int G = cfg->n_experts + cfg->n_shared;
+  int32_t* mt = reinterpret_cast<int32_t*>(ws + L.mt_prefix);
+  int32_t* mp = reinterpret_cast<int32_t*>(ws + L.mp_prefix);
+  CUDA_TRY(launch_tile_prefix(offsets, G, (int32_t)R, mt, mp, status, s));
+  if (stage == MOE_STAGE_DOWN) {
+    float* a_t = reinterpret_cast<float*>(ws + L.sh);
+    if (fp8) CUDA_TRY(launch_scale_transpose(a_scale, a_t, R, cfg->inter / 128, L.rows_pad, true, s));
+    return run_down(cfg, L, R, a, a_t, offsets, mt, mp, g_gemm_variant == MOE_GEMM_PAIR, w, row_gate, out, status, s);
+  }
+  float* a_t = reinterpret_cast<float*>(ws + L.sxp);
+  float* o_t = reinterpret_cast<float*>(ws + L.sh);
+  if (fp8) CUDA_TRY(launch_scale_transpose(a_scale, a_t, R, cfg->hidden / 128, L.rows_pad, true, s));
+  const bool raw = stage == MOE_STAGE_GATE_UP_RAW;
+  rc = run_gate_up(cfg, L, R, a, a_t, offsets, mt, mp, gate_up_on_pairs(R, G), w, out, o_t, raw, status, s);
+  if (rc != MOE_OK) return rc;
+  if (fp8 && !raw) CUDA_TRY(launch_scale_transpose(o_t, out_scale, R, cfg->inter / 128, L.rows_pad, false, s));
+  return MOE_OK;
+}
+
+int moe_read_status_detail(const void* workspace, moe_stream_t stream, int* detail) {
+  if (!workspace || !detail) return MOE_ERR_INVALID_ARG;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  int v[4] = {0, 0, 0, 0};
+  CUDA_TRY(cudaMemcpyAsync(v, workspace, sizeof(v), cudaMemcpyDeviceToHost, s));
+  CUDA_TRY(cudaStreamSynchronize(s));
+  for (int i = 0; i < 4; ++i) detail[i] = v[i];
+  return MOE_OK;
+}
+
+int moe_debug_inject(int what, uint64_t wait_limit_ns) {
+  if (what != MOE_INJECT_NONE && what != MOE_INJECT_GEMM_NO_LOADS) return MOE_ERR_INVALID_ARG;
+  g_inject = what;
+  g_wait_ns = wait_limit_ns ? wait_limit_ns : kWaitLimitNs;
+  return MOE_OK;
 }
 
 int moe_read_status(const void* workspace, moe_stream_t stream, int* device_status) {
@@ -580,6 +858,12 @@ const char* moe_profile_kernel_name(int i) { return (i >= 0 && i < kProfKernels)
 int moe_set_gemm_variant(int variant) {
   if (variant != MOE_GEMM_AUTO && variant != MOE_GEMM_SINGLE && variant != MOE_GEMM_PAIR) return MOE_ERR_INVALID_ARG;
   g_gemm_variant = variant;
+  return MOE_OK;
+}
+
+int moe_launch_count(uint64_t* n) {
+  if (!n) return MOE_ERR_INVALID_ARG;
+  *n = g_launches.load(std::memory_order_relaxed);
   return MOE_OK;
 }
 

@@ -16,6 +16,9 @@ constexpr int kStageBytesK = 128;    // K extent of one pipeline stage, in bytes
 constexpr int kHistChunk = 256;      // tokens per histogram/scatter CTA
 constexpr int kMaxExperts = 512;
 constexpr int kMaxTopK = 16;
+// Workspace status block: status word, first-timeout record (site, block,
+// progress), and the per-block counters of MOE_DEBUG_STATE builds.
+constexpr size_t kStatusBytes = 16384;
 
 __host__ __device__ inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 __host__ __device__ inline int64_t round_up(int64_t a, int64_t b) { return ceil_div(a, b) * b; }
@@ -53,6 +56,12 @@ struct TopkParams {
 // ---- histogram / scan / scatter ----
 struct PermuteParams {
   int32_t T, E, k, S, G, chunks;
+  // Expert parallelism: this call's groups are the routed experts
+  // [e0, e0 + E) of the E_all the routing chose from, and the shared expert's
+  // rows for tokens [sh_t0, sh_t1). Pairs routed to other experts are left out
+  // (pos = -1) without an error; an index outside [0, E_all) latches
+  // MOE_ERR_BAD_INDEX. One GPU: e0 = 0, E_all = E, [sh_t0, sh_t1) = [0, T).
+  int32_t e0, E_all, sh_t0, sh_t1;
   const int32_t* idx;       // [T, k]
   const float* gate;        // [T, k] or null (row gates then not written)
   int32_t* chunk_base;      // [E, chunks]: per-chunk counts, then absolute row bases
@@ -96,6 +105,9 @@ struct GemmParams {
   float* out_scale;          // GEMM1 FP8: [N/128, rows_pad]
   const float* row_gate;     // GEMM2: [R]
   int* status;
+  uint64_t wait_ns;          // limit of every bounded wait (normally 2 s)
+  int32_t raw_out;           // GEMM1 only: store the fp32 gate/up sums [R, 2N] instead of SwiGLU(h)
+  int32_t inject;            // test hook: 1 = the producer issues no loads (the first wait runs out)
 };
 
 struct CombineParams {
@@ -104,6 +116,10 @@ struct CombineParams {
   const int32_t* pos;        // [T, S]
   uint16_t* out;             // [T, H] bf16
 };
+
+// Counts a kernel launch of this library when `e` is cudaSuccess (read with
+// moe_launch_count) and returns `e`. Every launcher returns through it.
+cudaError_t counted_launch(cudaError_t e);
 
 // Host launchers (each returns the launch's cudaError_t).
 cudaError_t launch_router_gemm(const RouterParams& p, const CUtensorMap& tm_x, const CUtensorMap& tm_w,
@@ -125,6 +141,22 @@ struct AMaps {
   CUtensorMap rows128, rows64, rows32;
 };
 
+// NVFP4 weight tensor maps of one grouped GEMM (uint8, no swizzle): E2M1
+// codes [rows, K/2] with 32-byte boxes (one 64-deep K stage) and E4M3 scales
+// [rows, K/16] with 16-byte boxes (four stages). GEMM1: code0/scale0 = W1,
+// code1/scale1 = W3 (128-row boxes); GEMM2: code0/scale0 = W2 (256-row boxes).
+// The s-prefixed maps are the shared expert's.
+struct NvMaps {
+  CUtensorMap code0, code1, scode0, scode1, scale0, scale1, sscale0, sscale1;
+};
+
+// NVFP4 (W4A16) grouped GEMM, single CTAs: GEMM1 (gate/up + SwiGLU, bf16 h) or
+// GEMM2 (down, bf16 y). Global scales: GEMM1 b_scale0/b_scale1 = W1/W3 [E],
+// bs_scale0/bs_scale1 = the shared expert's [1]; GEMM2 b_scale0 = W2 [E],
+// bs_scale0 = the shared expert's.
+cudaError_t launch_nvfp4_gemm(const GemmParams& p, bool gemm1, int grid, const AMaps& tm_a, const NvMaps& tm,
+                              cudaStream_t s);
+
 cudaError_t launch_gemm1(const GemmParams& p, bool fp8, bool pair, int grid, const AMaps& tm_a,
                          const CUtensorMap& tm_w1, const CUtensorMap& tm_w3, const CUtensorMap& tm_sw1,
                          const CUtensorMap& tm_sw3, cudaStream_t s);
@@ -133,5 +165,15 @@ cudaError_t launch_gemm2(const GemmParams& p, bool fp8, bool pair, int grid, con
                          const CUtensorMap& tm_w2, const CUtensorMap& tm_w2h, const CUtensorMap& tm_sw2,
                          const CUtensorMap& tm_sw2h, cudaStream_t s);
 cudaError_t launch_combine(const CombineParams& p, cudaStream_t s);
+// Expert parallelism: a rank's fp32 partial output, the sum of each token's
+// expert rows that this rank computed (pos < 0 left out), in slot order.
+cudaError_t launch_ep_partial(int64_t T, int32_t H, int32_t S, const void* y, const int32_t* pos, float* part,
+                              cudaStream_t s);
+// Stage entry point helpers: tile prefixes of caller-given group offsets, and
+// FP8 scales between row-major [R, nb] and transposed [nb, rows_pad].
+cudaError_t launch_tile_prefix(const int32_t* offsets, int32_t G, int32_t R, int32_t* mt, int32_t* mp, int* status,
+                               cudaStream_t s);
+cudaError_t launch_scale_transpose(const float* src, float* dst, int64_t R, int32_t nb, int64_t rows_pad,
+                                   bool to_transposed, cudaStream_t s);
 
 }  // namespace moe

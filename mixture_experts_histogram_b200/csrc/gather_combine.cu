@@ -128,21 +128,41 @@ __global__ void __launch_bounds__(256) combine_kernel(const CombineParams p) {
   }
 }
 
+// FP8 activation scales between a caller's row-major [R, nb] layout and the
+// grouped GEMMs' transposed [nb, rows_pad] one (the stage entry point).
+__global__ void __launch_bounds__(256) scale_transpose_kernel(const float* __restrict__ src, float* __restrict__ dst,
+                                                              int64_t R, int32_t nb, int64_t rows_pad,
+                                                              int32_t to_transposed) {
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= R * nb) return;
+  const int64_t r = i / nb, kb = i % nb;
+  if (to_transposed) dst[kb * rows_pad + r] = src[i];
+  else dst[i] = src[kb * rows_pad + r];
+}
+
 }  // namespace
+
+cudaError_t launch_scale_transpose(const float* src, float* dst, int64_t R, int32_t nb, int64_t rows_pad,
+                                   bool to_transposed, cudaStream_t s) {
+  const int64_t n = R * nb;
+  if (n == 0) return cudaSuccess;
+  scale_transpose_kernel<<<(unsigned)ceil_div(n, 256), 256, 0, s>>>(src, dst, R, nb, rows_pad, to_transposed ? 1 : 0);
+  return counted_launch(cudaGetLastError());
+}
 
 cudaError_t launch_gather(const GatherParams& p, bool fp8, cudaStream_t s) {
   if (p.T == 0) return cudaSuccess;
   if (fp8 && p.S <= 9) gather_fp8_kernel<9><<<(unsigned)p.T, 256, 0, s>>>(p);
   else if (fp8) gather_fp8_kernel<kMaxTopK + 1><<<(unsigned)p.T, 256, 0, s>>>(p);
   else gather_bf16_kernel<<<(unsigned)p.T, 256, 0, s>>>(p);
-  return cudaGetLastError();
+  return counted_launch(cudaGetLastError());
 }
 
 cudaError_t launch_combine(const CombineParams& p, cudaStream_t s) {
   if (p.T == 0) return cudaSuccess;
   if (p.S <= 9) combine_kernel<9><<<(unsigned)p.T, 256, 0, s>>>(p);
   else combine_kernel<kMaxTopK + 1><<<(unsigned)p.T, 256, 0, s>>>(p);
-  return cudaGetLastError();
+  return counted_launch(cudaGetLastError());
 }
 
 }  // namespace moe

@@ -47,6 +47,7 @@
 #include <cuda_fp8.h>
 
 #include "common.cuh"
+#include "gemm_common.cuh"
 #include "ptx.cuh"
 
 namespace moe {
@@ -87,30 +88,6 @@ struct Cfg {
   static_assert(kDynamic <= 227 * 1024, "shared memory budget");
 };
 
-struct Item {
-  int g, n, row0, end;  // group, N tile, first row of the tile, end of the group's rows
-};
-
-// n_fastest: consecutive items walk the N tiles of one row tile (they share A
-// rows); otherwise they walk the M tiles of one weight tile (they share B).
-__device__ __forceinline__ Item decode_item(int item, int n_tiles, int G, int tile_rows, const int* s_mt,
-                                            const int* s_off, bool n_fastest) {
-  const int q = item / n_tiles;
-  int lo = 0, hi = G;  // s_mt[lo] <= q < s_mt[hi]
-  while (hi - lo > 1) {
-    const int mid = (lo + hi) >> 1;
-    if (s_mt[mid] <= q) lo = mid;
-    else hi = mid;
-  }
-  Item it;
-  it.g = lo;
-  const int mtiles = s_mt[lo + 1] - s_mt[lo];
-  const int local = item - n_tiles * s_mt[lo];
-  it.n = n_fastest ? local % n_tiles : local / mtiles;
-  it.row0 = s_off[lo] + (n_fastest ? local / n_tiles : local % mtiles) * tile_rows;
-  it.end = s_off[lo + 1];
-  return it;
-}
 
 // Weight-tile rows of a work item: box 0 starts at row `yb` of `*m0`, box 1 at
 // row `yb2` of `*m1`. GEMM1: W1 and W3 rows n0.. (128-row boxes). GEMM2: `*m0`
@@ -130,26 +107,6 @@ struct BRows {
   }
 };
 
-// silu(g) * u. The quotient uses the fast division: exact IEEE division falls
-// into its slow path whenever exp(-g) overflows (rows of a tile past its
-// group's end can hold large values), which once cost a fifth of GEMM1's time.
-// For an infinite denominator the fast quotient is 0, silu's limit.
-__device__ __forceinline__ float silu_mul(float g, float u) { return __fdividef(g, 1.0f + __expf(-g)) * u; }
-
-__device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
-  const __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
-  return *reinterpret_cast<const uint32_t*>(&v);
-}
-
-// Bounded wait by every lane, with a warp-uniform verdict (keeps the warp
-// converged for the .sync.aligned TMEM loads that follow).
-template <bool kCluster>
-__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, int* status, volatile int* abort_flag,
-                                          int site, int progress) {
-  const bool ok = kCluster ? mbar_wait_cluster(bar, parity, status, abort_flag, site, progress)
-                           : mbar_wait(bar, parity, status, abort_flag, site, progress);
-  return __all_sync(0xffffffffu, ok);
-}
 
 template <bool kFP8, bool kGemm1, bool kPair>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -246,7 +203,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t issued = 0;        // bit s: stage s has had a load issued
     uint32_t issued_phase = 0;  // bit s: the phase of that last issue
     bool ok = true;
-    for (int item = unit; item < total && ok; item += n_units) {
+    // (Test hook: with p.inject == 1 nothing is loaded, so the consumers' first
+    // waits run out and the kernel returns MOE_ERR_DEVICE_TIMEOUT with nothing
+    // in flight.)
+    for (int item = unit; item < total && ok && p.inject != 1; item += n_units) {
       const Item it = decode_item(item, p.n_tiles, p.G, C::kTileRows, s_mt, s_off, p.n_fastest != 0);
       const bool shared = (it.g == p.E);
       const int my_row0 = it.row0 + my_off;
@@ -278,7 +238,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int ks = 0; ks < kstages; ++ks) {
         bool w = true;
         MOE_DBG(item, ks, sc_iter);
-        if (lane == 0) w = mbar_wait(&empty[stage], phase ^ 1, p.status, abort_flag, site0 | 1, item);
+        if (lane == 0) w = mbar_wait(&empty[stage], phase ^ 1, p.status, abort_flag, site0 | 1, item, p.wait_ns);
         if (!__shfl_sync(0xffffffffu, w ? 1 : 0, 0)) { ok = false; break; }
         if (lane == 0) {
           const int kx = ks * kElemsPerStage;
@@ -306,7 +266,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (kFP8) {
           const uint32_t j = sc_iter % kScRing, sph = (sc_iter / kScRing) & 1u;
-          if (!warp_wait<false>(&scempty[j], sph ^ 1u, p.status, abort_flag, site0 | 2, item)) { ok = false; break; }
+          if (!warp_wait<false>(&scempty[j], sph ^ 1u, p.status, abort_flag, site0 | 2, item, p.wait_ns)) {
+            ok = false;
+            break;
+          }
           float* slot = sc + j * kScSlot;
           const float* src = p.a_scale + (int64_t)ks * p.rows_pad + my_row0 + lane * 4;
 #pragma unroll
@@ -347,8 +310,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         else mma_commit(bar);
       };
       auto wait_tempty = [&](uint32_t b, uint32_t par, uint32_t it) {
-        return kPair ? mbar_wait_cluster(&tempty[b], par, p.status, abort_flag, site0 | 3, (int)it)
-                     : mbar_wait(&tempty[b], par, p.status, abort_flag, site0 | 3, (int)it);
+        return kPair ? mbar_wait_cluster(&tempty[b], par, p.status, abort_flag, site0 | 3, (int)it, p.wait_ns)
+                     : mbar_wait(&tempty[b], par, p.status, abort_flag, site0 | 3, (int)it, p.wait_ns);
       };
       int stage = 0;
       uint32_t phase = 0;
@@ -361,7 +324,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_fence_after_sync();
           const uint32_t d = tmem + b * 256;
           for (int ks = 0; ks < kstages; ++ks) {
-            if (!mbar_wait(&full[stage], phase, p.status, abort_flag, site0 | 4, (int)acc_iter)) { ok = false; break; }
+            if (!mbar_wait(&full[stage], phase, p.status, abort_flag, site0 | 4, (int)acc_iter, p.wait_ns)) {
+              ok = false;
+              break;
+            }
             tc_fence_after_sync();
             const uint64_t ad = sdesc_k_sw128(sA + stage * kABytes);
             const uint64_t bd = sdesc_k_sw128(sB + stage * C::kBBytes);
@@ -378,7 +344,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t b = acc_iter & 1u, tph = (acc_iter >> 1) & 1u;
             MOE_DBG(item, ks, acc_iter);
             if (!wait_tempty(b, tph ^ 1u, acc_iter)) { ok = false; break; }
-            if (!mbar_wait(&full[stage], phase, p.status, abort_flag, site0 | 4, (int)acc_iter)) { ok = false; break; }
+            if (!mbar_wait(&full[stage], phase, p.status, abort_flag, site0 | 4, (int)acc_iter, p.wait_ns)) {
+              ok = false;
+              break;
+            }
             tc_fence_after_sync();
             const uint32_t d = tmem + b * 256;
             const uint64_t ad = sdesc_k_sw128(sA + stage * kABytes);
@@ -425,7 +394,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool col_ok = col0 < p.N;
       if (!kFP8) {
         const uint32_t b = acc_iter & 1u, tph = (acc_iter >> 1) & 1u;
-        if (ok) ok = warp_wait<false>(&tfull[b], tph, p.status, abort_flag, site0 | 6, (int)acc_iter);
+        if (ok) ok = warp_wait<false>(&tfull[b], tph, p.status, abort_flag, site0 | 6, (int)acc_iter, p.wait_ns);
         tc_fence_after_sync();
         const uint32_t base = tmem + lane_base + b * 256;
         if (kGemm1) {
@@ -436,6 +405,21 @@ __global__ void __launch_bounds__(kThreads, 1)
             tmem_ld32(base + 128 + 64 * hf + 32 * ch, u);
             tmem_ld_wait();
             if (ch == 1) release_acc(b);
+            if (p.raw_out) {
+              // The fp32 gate and up sums themselves (stage entry point, tests).
+              if (ok && row_ok) {
+                float4* dg = reinterpret_cast<float4*>(static_cast<float*>(p.out) + row * 2 * p.N + col0 + 32 * ch);
+                float4* du = dg + p.N / 4;
+#pragma unroll
+                for (int v = 0; v < 8; ++v) {
+                  dg[v] = make_float4(__uint_as_float(g[4 * v]), __uint_as_float(g[4 * v + 1]),
+                                      __uint_as_float(g[4 * v + 2]), __uint_as_float(g[4 * v + 3]));
+                  du[v] = make_float4(__uint_as_float(u[4 * v]), __uint_as_float(u[4 * v + 1]),
+                                      __uint_as_float(u[4 * v + 2]), __uint_as_float(u[4 * v + 3]));
+                }
+              }
+              continue;
+            }
             uint32_t pk[16];
 #pragma unroll
             for (int i = 0; i < 16; ++i)
@@ -448,7 +432,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
         } else {
-          const float gw = row_ok ? p.row_gate[row] : 0.0f;
+          const float gw = row_ok ? (p.row_gate ? p.row_gate[row] : 1.0f) : 0.0f;
 #pragma unroll
           for (int ch = 0; ch < 4; ++ch) {
             uint32_t v[32];
@@ -475,7 +459,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int kb = 0; kb < nkb; ++kb) {
           const uint32_t j = sc_iter % kScRing, sph = (sc_iter / kScRing) & 1u;
           MOE_DBG(item, kb, acc_iter);
-          if (ok) ok = warp_wait<false>(&scfull[j], sph, p.status, abort_flag, site0 | 5, (int)sc_iter);
+          if (ok) ok = warp_wait<false>(&scfull[j], sph, p.status, abort_flag, site0 | 5, (int)sc_iter, p.wait_ns);
           const float* slot = sc + j * kScSlot;
           const float a_s = slot[rl];
           const float s0 = slot[128], s1 = slot[129];
@@ -487,7 +471,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const float f0 = a_s * ((kGemm1 || hf == 0) ? s0 : s1);
           const float f1 = kGemm1 ? a_s * s1 : f0;
           const uint32_t b = acc_iter & 1u, tph = (acc_iter >> 1) & 1u;
-          if (ok) ok = warp_wait<false>(&tfull[b], tph, p.status, abort_flag, site0 | 6, (int)acc_iter);
+          if (ok) ok = warp_wait<false>(&tfull[b], tph, p.status, abort_flag, site0 | 6, (int)acc_iter, p.wait_ns);
           tc_fence_after_sync();
           const uint32_t base = tmem + lane_base + b * 256;
           constexpr int kNch = 128 / kFp8Chunk;  // chunks per thread per K block
@@ -532,7 +516,19 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           ++acc_iter;
         }
-        if (kGemm1) {
+        if (kGemm1 && p.raw_out) {
+          // The fp32 gate and up sums themselves (stage entry point, tests):
+          // acc[i] holds gate columns 2i, 2i+1 of this thread, acc[32 + i] the up ones.
+          if (ok && row_ok) {
+            float4* dg = reinterpret_cast<float4*>(static_cast<float*>(p.out) + row * 2 * p.N + col0);
+            float4* du = dg + p.N / 4;
+#pragma unroll
+            for (int v = 0; v < 16; ++v) {
+              dg[v] = make_float4(acc[2 * v].x, acc[2 * v].y, acc[2 * v + 1].x, acc[2 * v + 1].y);
+              du[v] = make_float4(acc[32 + 2 * v].x, acc[32 + 2 * v].y, acc[33 + 2 * v].x, acc[33 + 2 * v].y);
+            }
+          }
+        } else if (kGemm1) {
           // SwiGLU in place (acc[0..31] gate, acc[32..63] up), then the 1x128 block
           // quantisation of h; the block spans both column halves.
           float amax = 0.0f;
@@ -565,7 +561,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           ++tile_iter;
         } else {
-          const float gw = row_ok ? p.row_gate[row] : 0.0f;
+          const float gw = row_ok ? (p.row_gate ? p.row_gate[row] : 1.0f) : 0.0f;
           if (ok && row_ok && col_ok) {
             uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.out) + row * p.N + col0);
 #pragma unroll
@@ -580,8 +576,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   }
 #ifdef MOE_DEBUG_STATE
-  // Debug builds: each role's final counters, 16 ints per block from status[64].
-  if (kGemm1 && lane == 0 && blockIdx.x < 900) {
+  // Debug builds: each role's final counters, 16 ints per block from status[64],
+  // for the blocks whose counters fit in the workspace's status block.
+  constexpr unsigned kDbgBlocks = (unsigned)((kStatusBytes / 4 - 64) / 16);
+  static_assert(64 + kDbgBlocks * 16 <= kStatusBytes / 4, "debug counters overrun the status block");
+  if (kGemm1 && lane == 0 && blockIdx.x < kDbgBlocks) {
     int* dbg = p.status + 64 + blockIdx.x * 16;
     if (warp == 0) { dbg[0] = dbg_a; dbg[1] = dbg_b; dbg[2] = dbg_c; }
     if (warp == 1) { dbg[3] = dbg_a; dbg[4] = dbg_b; dbg[5] = dbg_c; }
@@ -613,7 +612,7 @@ cudaError_t launch_one(const GemmParams& p, int grid, const AMaps& a, const CUte
   }
   if (!kPair) {
     kern<<<grid, kThreads, Cfg<kPair>::kDynamic, s>>>(p, a, b0, b1, bs0, bs1);
-    return cudaGetLastError();
+    return counted_launch(cudaGetLastError());
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)(grid & ~1));
@@ -627,7 +626,7 @@ cudaError_t launch_one(const GemmParams& p, int grid, const AMaps& a, const CUte
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kern, p, a, b0, b1, bs0, bs1);
+  return counted_launch(cudaLaunchKernelEx(&cfg, kern, p, a, b0, b1, bs0, bs1));
 }
 
 }  // namespace

@@ -90,6 +90,10 @@ extern "C" int moe_permute_noalloc(const moe_config* cfg, int64_t T, const int32
   pp.k = cfg->top_k;
   pp.S = cfg->n_shared;
   pp.G = G;
+  pp.e0 = 0;
+  pp.E_all = cfg->n_experts;
+  pp.sh_t0 = 0;
+  pp.sh_t1 = (int32_t)T;
   pp.chunks = (int32_t)chunks;
   pp.idx = topk_idx;
   pp.gate = nullptr;

@@ -35,9 +35,9 @@ __device__ __forceinline__ void histogram_block(const PermuteParams& p, int chun
   const int64_t npairs = ntok * p.k;
   const int32_t* idx = p.idx + t0 * p.k;
   for (int64_t i = threadIdx.x; i < npairs; i += blockDim.x) {
-    const int e = idx[i];
-    if (e < 0 || e >= p.E) latch_status(p.status, MOE_ERR_BAD_INDEX);
-    else atomicAdd(&cnt[e], 1);
+    const int eg = idx[i], e = eg - p.e0;
+    if (eg < 0 || eg >= p.E_all) latch_status(p.status, MOE_ERR_BAD_INDEX);
+    else if (e >= 0 && e < p.E) atomicAdd(&cnt[e], 1);
   }
   __syncthreads();
   for (int e = threadIdx.x; e < p.E; e += blockDim.x) p.chunk_base[(int64_t)e * p.chunks + chunk] = cnt[e];
@@ -72,7 +72,7 @@ __device__ __forceinline__ void scan_block(const PermuteParams& p, int* cnt_s, i
     }
     if (lane == 0) cnt_s[e] = running;
   }
-  if (threadIdx.x == 0 && p.S) cnt_s[p.E] = p.T;
+  if (threadIdx.x == 0 && p.S) cnt_s[p.E] = p.sh_t1 - p.sh_t0;
   __syncthreads();
   // offsets and M-tile prefix over the G groups
   if (warp == 0) {
@@ -132,8 +132,8 @@ __device__ __forceinline__ void scatter_block(const PermuteParams& p, int chunk,
       const int j = pidx % p.k;
       int e = -1;
       if (t < p.T) {
-        e = p.idx[t * p.k + j];
-        if (e < 0 || e >= p.E) e = -1;
+        e = p.idx[t * p.k + j] - p.e0;  // this call's group; others are left out
+        if (e < 0 || e >= p.E || e + p.e0 >= p.E_all) e = -1;
       }
       const int key = e >= 0 ? e : (0x40000000 + lane);  // unmatched sentinel for empty lanes
       const unsigned m = __match_any_sync(0xffffffffu, key);
@@ -174,19 +174,23 @@ __device__ __forceinline__ void scatter_block(const PermuteParams& p, int chunk,
           p.pos[t * S + j] = row;
           if (p.row_gate) p.row_gate[row] = p.gate[t * p.k + j];
         } else {
-          p.pos[t * S + j] = -1;  // a skipped (bad-index) pair
+          p.pos[t * S + j] = -1;  // a pair left out (another rank's expert, or a bad index)
         }
       }
     }
   }
-  // The shared expert's rows: token order.
+  // The shared expert's rows: token order, for tokens [sh_t0, sh_t1).
   if (p.S) {
     const int64_t t = (int64_t)chunk * kHistChunk + threadIdx.x;
     if (t < p.T) {
-      const int row = p.offsets[p.E] + (int)t;
-      p.perm[row] = (int32_t)t;
-      p.pos[t * S + p.k] = row;
-      if (p.row_gate) p.row_gate[row] = 1.0f;
+      if (t >= p.sh_t0 && t < p.sh_t1) {
+        const int row = p.offsets[p.E] + (int)(t - p.sh_t0);
+        p.perm[row] = (int32_t)t;
+        p.pos[t * S + p.k] = row;
+        if (p.row_gate) p.row_gate[row] = 1.0f;
+      } else {
+        p.pos[t * S + p.k] = -1;
+      }
     }
   }
 }
@@ -208,16 +212,16 @@ __global__ void __launch_bounds__(256) permute_one_chunk_kernel(const PermutePar
   __syncthreads();
   const int npairs = p.T * p.k;
   for (int i = threadIdx.x; i < npairs; i += blockDim.x) {
-    const int e = p.idx[i];
-    if (e < 0 || e >= p.E) latch_status(p.status, MOE_ERR_BAD_INDEX);
-    else atomicAdd(&cnt[e], 1);
+    const int eg = p.idx[i], e = eg - p.e0;
+    if (eg < 0 || eg >= p.E_all) latch_status(p.status, MOE_ERR_BAD_INDEX);
+    else if (e >= 0 && e < p.E) atomicAdd(&cnt[e], 1);
   }
   __syncthreads();
   if (warp == 0) {
     int run_off = 0, run_mt = 0, run_mp = 0;
     for (int g0 = 0; g0 < p.G; g0 += 32) {
       const int g = g0 + lane;
-      const int c = g < p.E ? cnt[g] : (g < p.G ? p.T : 0);  // group E: the shared expert
+      const int c = g < p.E ? cnt[g] : (g < p.G ? p.sh_t1 - p.sh_t0 : 0);  // group E: the shared expert
       const int mt = (c + kTileM - 1) / kTileM;
       const int mp = (c + 2 * kTileM - 1) / (2 * kTileM);
       const int ic = warp_inclusive_scan(c, lane);
@@ -244,26 +248,64 @@ __global__ void __launch_bounds__(256) permute_one_chunk_kernel(const PermutePar
   scatter_block(p, 0, wcnt);
 }
 
+// Tile prefixes of caller-given group offsets (the grouped-GEMM stage entry
+// point), one warp. The offsets must start at 0, never decrease and end at most
+// at R; otherwise MOE_ERR_INVALID_ARG is latched and every group gets zero
+// tiles, so the GEMM that follows touches nothing.
+__global__ void __launch_bounds__(32) tile_prefix_kernel(const int32_t* offsets, int32_t G, int32_t R, int32_t* mt,
+                                                         int32_t* mp, int* status) {
+  const int lane = threadIdx.x;
+  bool bad = lane == 0 && (offsets[0] != 0 || offsets[G] > R);
+  for (int g = lane; g < G; g += 32) bad = bad || offsets[g + 1] < offsets[g];
+  bad = __any_sync(0xffffffffu, bad);
+  if (bad) latch_status(status, MOE_ERR_INVALID_ARG);
+  int run_mt = 0, run_mp = 0;
+  for (int g0 = 0; g0 < G; g0 += 32) {
+    const int g = g0 + lane;
+    const int c = (g < G && !bad) ? offsets[g + 1] - offsets[g] : 0;
+    const int t1 = (c + kTileM - 1) / kTileM;
+    const int t2 = (c + 2 * kTileM - 1) / (2 * kTileM);
+    const int i1 = warp_inclusive_scan(t1, lane);
+    const int i2 = warp_inclusive_scan(t2, lane);
+    if (g < G) {
+      mt[g] = run_mt + i1 - t1;
+      mp[g] = run_mp + i2 - t2;
+    }
+    run_mt += __shfl_sync(0xffffffffu, i1, 31);
+    run_mp += __shfl_sync(0xffffffffu, i2, 31);
+  }
+  if (lane == 0) {
+    mt[G] = run_mt;
+    mp[G] = run_mp;
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_tile_prefix(const int32_t* offsets, int32_t G, int32_t R, int32_t* mt, int32_t* mp, int* status,
+                               cudaStream_t s) {
+  tile_prefix_kernel<<<1, 32, 0, s>>>(offsets, G, R, mt, mp, status);
+  return counted_launch(cudaGetLastError());
+}
 
 cudaError_t launch_permute_one_chunk(const PermuteParams& p, cudaStream_t s) {
   permute_one_chunk_kernel<<<1, 256, 0, s>>>(p);
-  return cudaGetLastError();
+  return counted_launch(cudaGetLastError());
 }
 
 cudaError_t launch_histogram(const PermuteParams& p, cudaStream_t s) {
   histogram_kernel<<<p.chunks, 256, 0, s>>>(p);
-  return cudaGetLastError();
+  return counted_launch(cudaGetLastError());
 }
 
 cudaError_t launch_scan(const PermuteParams& p, cudaStream_t s) {
   scan_kernel<<<1, 1024, 0, s>>>(p);
-  return cudaGetLastError();
+  return counted_launch(cudaGetLastError());
 }
 
 cudaError_t launch_scatter(const PermuteParams& p, cudaStream_t s) {
   scatter_kernel<<<p.chunks, 256, 0, s>>>(p);
-  return cudaGetLastError();
+  return counted_launch(cudaGetLastError());
 }
 
 }  // namespace moe

@@ -12,7 +12,9 @@
 namespace moe {
 
 // A wait gives up after this long and latches MOE_ERR_DEVICE_TIMEOUT, so a
-// protocol error ends the kernel with an error status instead of a hang.
+// protocol error ends the kernel with an error status instead of a hang. The
+// expert GEMMs take their limit from their parameters (moe_debug_inject can
+// shorten it for a test); every other kernel uses this one.
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -72,9 +74,10 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 
 // Waits for the phase of `bar` with the given parity to complete. Returns
 // false (and latches a timeout, and raises the CTA's abort flag) if it does not
-// complete within kWaitLimitNs, or if another role of the CTA already aborted.
+// complete within limit_ns, or if another role of the CTA already aborted.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* status,
-                                          volatile int* abort_flag, int site = 0, int progress = 0) {
+                                          volatile int* abort_flag, int site = 0, int progress = 0,
+                                          uint64_t limit_ns = kWaitLimitNs) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
   uint32_t spins = 0;
@@ -82,7 +85,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* s
     if (mbar_try_wait(bar, parity)) return true;
     if ((++spins & 63u) == 0) {
       if (*abort_flag) return false;
-      if (global_timer_ns() - t0 > kWaitLimitNs) {
+      if (global_timer_ns() - t0 > limit_ns) {
         latch_timeout(status, site, progress);
         *abort_flag = 1;
         return false;
@@ -192,7 +195,8 @@ __device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t pa
 
 // Bounded wait with cluster-scope acquire (for barriers that peer CTAs arrive on).
 __device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity, int* status,
-                                                  volatile int* abort_flag, int site = 0, int progress = 0) {
+                                                  volatile int* abort_flag, int site = 0, int progress = 0,
+                                                  uint64_t limit_ns = kWaitLimitNs) {
   if (mbar_try_wait_cluster(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
   uint32_t spins = 0;
@@ -200,7 +204,7 @@ __device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity
     if (mbar_try_wait_cluster(bar, parity)) return true;
     if ((++spins & 63u) == 0) {
       if (*abort_flag) return false;
-      if (global_timer_ns() - t0 > kWaitLimitNs) {
+      if (global_timer_ns() - t0 > limit_ns) {
         latch_timeout(status, site, progress);
         *abort_flag = 1;
         return false;

@@ -111,7 +111,7 @@ extern "C" int moe_rmsnorm(int64_t T, int32_t hidden, const float* residual, con
   if (!aligned16(residual) || !aligned16(weight) || !aligned16(x_bf16)) return MOE_ERR_MISALIGNED;
   rmsnorm_kernel<<<(unsigned)T, kThreads, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
       hidden, residual, weight, eps, static_cast<uint16_t*>(x_bf16));
-  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+  return counted_launch(cudaGetLastError()) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
 extern "C" int moe_combine_residual(const moe_config* cfg, int64_t T, const void* y, const int32_t* pos,
@@ -131,5 +131,5 @@ extern "C" int moe_combine_residual(const moe_config* cfg, int64_t T, const void
   else
     combine_residual_kernel<kMaxTopK + 1><<<(unsigned)T, kThreads, 0, s>>>(
         cfg->hidden, S, static_cast<const uint16_t*>(y), pos, residual, residual_out);
-  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+  return counted_launch(cudaGetLastError()) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }

@@ -250,12 +250,12 @@ cudaError_t launch_router_gemm(const RouterParams& p, const CUtensorMap& tm_x, c
   if (e != cudaSuccess) return e;
   dim3 grid((unsigned)ceil_div(p.T, kTileM), (unsigned)p.ksplit);
   router_gemm_kernel<<<grid, kRouterThreads, smem, s>>>(p, tm_x, tm_w);
-  return cudaGetLastError();
+  return counted_launch(cudaGetLastError());
 }
 
 cudaError_t launch_topk(const TopkParams& p, cudaStream_t s) {
   topk_kernel<<<(unsigned)ceil_div(p.T, 8), 256, 0, s>>>(p);
-  return cudaGetLastError();
+  return counted_launch(cudaGetLastError());
 }
 
 }  // namespace moe

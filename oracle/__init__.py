@@ -11,12 +11,20 @@ Functions and the passages they follow:
                    "Step-5-Preview" page, "Model Architecture" table)
   quantize_rows    1x128 E4M3 activation blocks (StepFun "Step-5 minimal
                    inference" README: block-scaled FP8 expert GEMM)
+  e2m1_decode, nvfp4_dequantize
+                   NVFP4 weights: E2M1 codes two to a byte, an E4M3 scale per
+                   16 inputs, an fp32 global scale (TensorFold PR page, the
+                   NVFP4 format of its W4A16 linears)
   permute          token->expert histogram, exclusive scan and gather indices
                    (README: the "critical MoE primitives")
   moe_tokens       expert SwiGLU MLPs and the weighted combine, fp64 sums in
                    slot order (README, "Long-output stability": fixed-order
                    accumulation in at least fp32)
+  expert_rows      single (token, expert) output rows, the per-row evaluation
+                   of moe_tokens (same README row)
   moe_forward      route + moe_tokens for a whole batch (or a token sample)
+  ep_partial       one expert-parallel rank's share of the output (README,
+                   deployment at TP = EP and "Long-output stability")
   rmsnorm          the fp32 residual stream normalised into the layer's bf16
                    input (NeMo "Step-5-Preview" page, "Full-Depth H100
                    Benchmark" table: FP32 norms and residuals)
@@ -47,7 +55,7 @@ class _Shape(ctypes.Structure):
 class _Weights(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in
                 ("router_w", "router_bias", "w1", "w3", "w2", "s1", "s3", "s2",
-                 "sw1", "sw3", "sw2", "ss1", "ss3", "ss2")]
+                 "sw1", "sw3", "sw2", "ss1", "ss3", "ss2", "g1", "g3", "g2", "sg1", "sg3", "sg2")]
 
 
 def build(force: bool = False) -> str:
@@ -68,6 +76,8 @@ def _load():
         lib.orc_num_threads.restype = ctypes.c_int
         lib.orc_e4m3_value.argtypes = [ctypes.c_uint8]
         lib.orc_e4m3_value.restype = ctypes.c_double
+        lib.orc_e2m1_value.argtypes = [ctypes.c_uint8]
+        lib.orc_e2m1_value.restype = ctypes.c_double
         lib.orc_e4m3_encode.argtypes = [ctypes.c_float]
         lib.orc_e4m3_encode.restype = ctypes.c_uint8
         lib.orc_e4m3_encode_array.argtypes = [i64, vp, vp]
@@ -78,6 +88,7 @@ def _load():
         lib.orc_permute.restype = ctypes.c_int
         lib.orc_moe_tokens.argtypes = [ctypes.POINTER(_Shape), ctypes.POINTER(_Weights), vp, vp, vp, i64, vp,
                                        vp, vp, vp]
+        lib.orc_expert_rows.argtypes = [ctypes.POINTER(_Shape), ctypes.POINTER(_Weights), vp, i64, vp, vp, vp]
         _lib = lib
     return _lib
 
@@ -102,6 +113,24 @@ def e4m3_decode(codes: np.ndarray) -> np.ndarray:
     out = np.empty(c.shape, dtype=np.float64)
     _load().orc_e4m3_decode_array(c.size, _p(c), _p(out))
     return out
+
+
+def e2m1_decode(codes: np.ndarray) -> np.ndarray:
+    """Exact values (float64) of 4-bit E2M1 codes (the low nibble of each uint8)."""
+    c = np.asarray(codes, dtype=np.uint8) & 15
+    lib = _load()
+    table = np.array([lib.orc_e2m1_value(i) for i in range(16)], dtype=np.float64)
+    return table[c]
+
+
+def nvfp4_dequantize(codes: np.ndarray, scales: np.ndarray, global_scale: float) -> np.ndarray:
+    """One NVFP4 matrix: codes [n, k/2] (input 2j in byte j's low nibble),
+    E4M3 scales [n, k/16], global fp32 scale -> float64 [n, k]."""
+    lo = e2m1_decode(codes & 15)
+    hi = e2m1_decode(codes >> 4)
+    v = np.stack([lo, hi], axis=-1).reshape(codes.shape[0], codes.shape[1] * 2)
+    s = np.repeat(e4m3_decode(scales), 16, axis=1)
+    return v * s * float(global_scale)
 
 
 def e4m3_encode(values: np.ndarray) -> np.ndarray:
@@ -195,6 +224,27 @@ def moe_tokens(shape, weights: dict, x_bf16: np.ndarray, idx: np.ndarray, gate: 
     return out, outb, y
 
 
+def expert_rows(shape, weights: dict, x_bf16: np.ndarray, tokens: Sequence[int], groups: Sequence[int]):
+    """Ungated output rows y [n, H] (f64) of group groups[i] on token tokens[i].
+
+    Groups 0..E-1 are the routed experts and group E the shared expert; the
+    same per-row evaluation as moe_tokens, for chosen rows of a large batch.
+    """
+    x = np.ascontiguousarray(x_bf16, dtype=np.uint16)
+    T, H = x.shape
+    toks = np.ascontiguousarray(tokens, dtype=np.int64)
+    grp = np.ascontiguousarray(groups, dtype=np.int32)
+    assert toks.shape == grp.shape and toks.ndim == 1
+    assert np.all((toks >= 0) & (toks < T)) and np.all((grp >= 0) & (grp <= shape.n_experts))
+    assert shape.n_shared == 1 or np.all(grp < shape.n_experts)
+    sh = _Shape(T, shape.hidden, shape.n_experts, shape.top_k, shape.n_shared, shape.inter, shape.wdtype)
+    ws, keep = _weights_struct(weights)
+    y = np.empty((toks.size, H), dtype=np.float64)
+    _load().orc_expert_rows(ctypes.byref(sh), ctypes.byref(ws), _p(x), toks.size, _p(toks), _p(grp), _p(y))
+    del keep
+    return y
+
+
 def moe_forward(shape, weights: dict, x_bf16: np.ndarray, tokens: Optional[Sequence[int]] = None):
     """Whole layer: routing for every token, outputs for `tokens` (default all).
 
@@ -204,6 +254,30 @@ def moe_forward(shape, weights: dict, x_bf16: np.ndarray, tokens: Optional[Seque
                               want_logits=True)
     out, outb, _ = moe_tokens(shape, weights, x_bf16, idx, gate, tokens)
     return {"idx": idx, "gate": gate, "logits": logits, "out_f64": out, "out_bf16": outb}
+
+
+# ------------------------------------------------------ expert parallelism --
+
+def ep_partial(shape, weights: dict, x_bf16: np.ndarray, idx: np.ndarray, gate: np.ndarray, e0: int, e1: int,
+               t0: int, t1: int, tokens: Optional[Sequence[int]] = None) -> np.ndarray:
+    """One expert-parallel rank's share of the output, fp64 [n, H]: for each
+    token, the gate-weighted rows of its routed experts inside [e0, e1), in
+    slot order, plus its shared-expert row if the token lies in [t0, t1)
+    (StepFun README, deployment at TP = EP: each rank holds a range of the
+    routed experts; the ranks' partial results are added in rank order).
+    Summed over ranks whose ranges partition the experts and the tokens, the
+    partials give moe_tokens' output."""
+    toks = np.arange(x_bf16.shape[0], dtype=np.int64) if tokens is None else np.asarray(tokens, dtype=np.int64)
+    _, _, y = moe_tokens(shape, weights, x_bf16, idx, gate, tokens=toks, want_y=True)
+    k = shape.top_k
+    out = np.zeros((toks.size, shape.hidden), dtype=np.float64)
+    for n, t in enumerate(toks):
+        for j in range(k):
+            if e0 <= idx[t, j] < e1:
+                out[n] += float(gate[t, j]) * y[n, j]
+        if shape.n_shared and t0 <= t < t1:
+            out[n] += y[n, k]
+    return out
 
 
 # ---------------------------------------------------------- residual stream --

@@ -15,7 +15,10 @@
  *
  *   Expert storage -- StepFun "Step-5 minimal inference" README, opening section
  *   and the expert-storage paragraph before "Install": experts are BF16, or FP8
- *   E4M3 with block scales ("block-scaled FP8 expert GEMM").
+ *   E4M3 with block scales ("block-scaled FP8 expert GEMM"). A third storage,
+ *   NVFP4 (TensorFold PR page: E2M1 codes, an E4M3 scale per 16 inputs and an
+ *   fp32 global scale, read by W4A16 linears), is a variant the pages describe
+ *   for another model; it keeps the BF16 activations.
  *
  *   Accumulation -- same README, "Long-output stability": partial results are
  *   added in a fixed order with FP32 (here: at least FP32) accumulation.
@@ -263,46 +266,75 @@ int orc_permute(int64_t T, int32_t E, int32_t k, int32_t n_shared, const int32_t
 
 /* ---------------------------------------------------------- expert MLPs ---- */
 
+/* ---------------------------------------------------------------- NVFP4 ---- */
+/*
+ * NVFP4 expert storage, as the TensorFold PR page describes the format its
+ * W4A16 linears read: E2M1 codes two to a byte (input 2j in the low nibble of
+ * byte j), one E4M3 scale per 16 inputs, and an fp32 global scale that
+ * multiplies; an element is e2m1 x e4m3 x global. E2M1 (OCP 4-bit float): one
+ * sign bit, two exponent bits with bias 1 and one mantissa bit; exponent 0 is
+ * subnormal (m x 0.5). Its magnitudes are 0, 0.5, 1, 1.5, 2, 3, 4 and 6.
+ */
+double orc_e2m1_value(uint8_t code) {
+  const int s = (code >> 3) & 1, e = (code >> 1) & 3, m = code & 1;
+  const double mag = (e == 0) ? 0.5 * m : ldexp(1.0 + 0.5 * m, e - 1);
+  return s ? -mag : mag;
+}
+
+/* ---------------------------------------------------------- expert MLPs ---- */
+
+/* wdtype: 0 = BF16; 1 = FP8 E4M3 with 128x128 fp32 block scales (E4M3 1x128
+ * activations); 2 = NVFP4 (bf16 activations and h, as for BF16). */
 typedef struct {
   int64_t T;
-  int32_t H, E, k, n_shared, I, wdtype; /* wdtype: 0 = BF16, 1 = FP8 E4M3 + 128x128 fp32 scales */
+  int32_t H, E, k, n_shared, I, wdtype;
 } orc_shape;
 
 typedef struct {
   const uint16_t* router_w;
   const float* router_bias;
-  const void *w1, *w3, *w2;          /* [E, I, H], [E, I, H], [E, H, I] */
-  const float *s1, *s3, *s2;         /* [E, I/128, H/128], [E, I/128, H/128], [E, H/128, I/128] */
-  const void *sw1, *sw3, *sw2;       /* shared expert, same layouts with E = 1 */
-  const float *ss1, *ss3, *ss2;
+  const void *w1, *w3, *w2;   /* [E, I, H], [E, I, H], [E, H, I]; NVFP4: codes [E, I, H/2], [E, I, H/2], [E, H, I/2] */
+  const void *s1, *s3, *s2;   /* FP8: fp32 [E, I/128, H/128], .., [E, H/128, I/128]; NVFP4: E4M3 [E, I, H/16], .., [E, H, I/16] */
+  const void *sw1, *sw3, *sw2; /* shared expert, same layouts with E = 1 */
+  const void *ss1, *ss3, *ss2;
+  const float *g1, *g3, *g2;    /* NVFP4 global scales [E] */
+  const float *sg1, *sg3, *sg2; /* NVFP4 global scales of the shared expert [1] */
 } orc_weights;
 
 /* Weight element W[g][r][c] of a stacked [G, R, C] tensor, dequantised exactly. */
-static double wval(const orc_shape* sh, const void* w, const float* s, int64_t g, int64_t R, int64_t C,
-                   int64_t r, int64_t c) {
-  const int64_t i = (g * R + r) * C + c;
-  if (sh->wdtype == 0) return bf16_val(((const uint16_t*)w)[i]);
-  const double sc = (double)s[(g * (R / 128) + r / 128) * (C / 128) + c / 128];
-  return orc_e4m3_value(((const uint8_t*)w)[i]) * sc;
+static double wval(const orc_shape* sh, const void* w, const void* s, const float* gs, int64_t g, int64_t R,
+                   int64_t C, int64_t r, int64_t c) {
+  const int64_t row = g * R + r;
+  if (sh->wdtype == 0) return bf16_val(((const uint16_t*)w)[row * C + c]);
+  if (sh->wdtype == 1) {
+    const double sc = (double)((const float*)s)[(g * (R / 128) + r / 128) * (C / 128) + c / 128];
+    return orc_e4m3_value(((const uint8_t*)w)[row * C + c]) * sc;
+  }
+  const uint8_t byte = ((const uint8_t*)w)[row * (C / 2) + c / 2];
+  const uint8_t code = (c & 1) ? (uint8_t)(byte >> 4) : (uint8_t)(byte & 15);
+  const uint8_t scale = ((const uint8_t*)s)[row * (C / 16) + c / 16];
+  return orc_e2m1_value(code) * orc_e4m3_value(scale) * (double)gs[g];
 }
 
 /*
  * One expert on one activation row a[H] (already the values the expert sees):
  * y[H] = (round_h(silu(a W1^T) * (a W3^T))) W2^T, sums in double.
  */
-static void expert_row(const orc_shape* sh, const void* w1, const float* s1, const void* w3,
-                       const float* s3, const void* w2, const float* s2, int64_t g, const double* a,
+static void expert_row(const orc_shape* sh, const orc_weights* w, int shared, int64_t g, const double* a,
                        double* hbuf, float* hf, uint8_t* hq, float* hs, double* y) {
   const int64_t H = sh->H, I = sh->I;
+  const void *w1 = shared ? w->sw1 : w->w1, *w3 = shared ? w->sw3 : w->w3, *w2 = shared ? w->sw2 : w->w2;
+  const void *s1 = shared ? w->ss1 : w->s1, *s3 = shared ? w->ss3 : w->s3, *s2 = shared ? w->ss2 : w->s2;
+  const float *g1 = shared ? w->sg1 : w->g1, *g3 = shared ? w->sg3 : w->g3, *g2 = shared ? w->sg2 : w->g2;
   for (int64_t i = 0; i < I; ++i) {
     double gt = 0.0, up = 0.0;
     for (int64_t h = 0; h < H; ++h) {
-      gt += a[h] * wval(sh, w1, s1, g, I, H, i, h);
-      up += a[h] * wval(sh, w3, s3, g, I, H, i, h);
+      gt += a[h] * wval(sh, w1, s1, g1, g, I, H, i, h);
+      up += a[h] * wval(sh, w3, s3, g3, g, I, H, i, h);
     }
     hbuf[i] = gt / (1.0 + exp(-gt)) * up; /* silu(gate) * up */
   }
-  if (sh->wdtype == 0) {
+  if (sh->wdtype != 1) {
     for (int64_t i = 0; i < I; ++i) hbuf[i] = bf16_val(float_to_bf16((float)hbuf[i]));
   } else {
     for (int64_t i = 0; i < I; ++i) hf[i] = (float)hbuf[i];
@@ -311,7 +343,7 @@ static void expert_row(const orc_shape* sh, const void* w1, const float* s1, con
   }
   for (int64_t c = 0; c < H; ++c) {
     double acc = 0.0;
-    for (int64_t i = 0; i < I; ++i) acc += hbuf[i] * wval(sh, w2, s2, g, H, I, c, i);
+    for (int64_t i = 0; i < I; ++i) acc += hbuf[i] * wval(sh, w2, s2, g2, g, H, I, c, i);
     y[c] = acc;
   }
 }
@@ -344,7 +376,7 @@ void orc_moe_tokens(const orc_shape* sh, const orc_weights* w, const uint16_t* x
     for (int64_t pi = 0; pi < n_tok * S; ++pi) {
       const int64_t n = pi / S, j = pi % S, t = tokens[n];
       /* the activation row the experts see */
-      if (sh->wdtype == 0) {
+      if (sh->wdtype != 1) {
         for (int64_t h = 0; h < H; ++h) a[h] = bf16_val(x[t * H + h]);
       } else {
         for (int64_t h = 0; h < H; ++h) xf[h] = (float)bf16_val(x[t * H + h]);
@@ -352,11 +384,8 @@ void orc_moe_tokens(const orc_shape* sh, const orc_weights* w, const uint16_t* x
         for (int64_t h = 0; h < H; ++h) a[h] = orc_e4m3_value(xq[h]) * (double)xs[h / 128];
       }
       double* y = ys + pi * H;
-      if (j < k) {
-        expert_row(sh, w->w1, w->s1, w->w3, w->s3, w->w2, w->s2, idx[t * k + j], a, hbuf, hf, hq, hs, y);
-      } else {
-        expert_row(sh, w->sw1, w->ss1, w->sw3, w->ss3, w->sw2, w->ss2, 0, a, hbuf, hf, hq, hs, y);
-      }
+      if (j < k) expert_row(sh, w, 0, idx[t * k + j], a, hbuf, hf, hq, hs, y);
+      else expert_row(sh, w, 1, 0, a, hbuf, hf, hq, hs, y);
     }
     free(a); free(hbuf); free(hf); free(hq); free(hs); free(xf); free(xq); free(xs);
   }
@@ -372,4 +401,42 @@ void orc_moe_tokens(const orc_shape* sh, const orc_weights* w, const uint16_t* x
   }
   if (y_out) memcpy(y_out, ys, sizeof(double) * (size_t)(n_tok * S * H));
   free(ys);
+}
+
+/*
+ * Single expert rows: y_out[i] = the (ungated) output of group groups[i] on
+ * token tokens[i]'s activation row, for i < n. Groups 0..E-1 are the routed
+ * experts, group E the shared expert. The same per-row evaluation as
+ * orc_moe_tokens, for checking chosen rows of a large batch one by one.
+ */
+void orc_expert_rows(const orc_shape* sh, const orc_weights* w, const uint16_t* x, int64_t n,
+                     const int64_t* tokens, const int32_t* groups, double* y_out) {
+  e4m3_init();
+  const int64_t H = sh->H, I = sh->I;
+#pragma omp parallel
+  {
+    double* a = (double*)malloc(sizeof(double) * (size_t)H);
+    double* hbuf = (double*)malloc(sizeof(double) * (size_t)I);
+    float* hf = (float*)malloc(sizeof(float) * (size_t)I);
+    uint8_t* hq = (uint8_t*)malloc((size_t)I);
+    float* hs = (float*)malloc(sizeof(float) * (size_t)(I / 128));
+    float* xf = (float*)malloc(sizeof(float) * (size_t)H);
+    uint8_t* xq = (uint8_t*)malloc((size_t)H);
+    float* xs = (float*)malloc(sizeof(float) * (size_t)(H / 128));
+#pragma omp for schedule(dynamic, 1)
+    for (int64_t i = 0; i < n; ++i) {
+      const int64_t t = tokens[i];
+      const int g = groups[i];
+      if (sh->wdtype != 1) {
+        for (int64_t h = 0; h < H; ++h) a[h] = bf16_val(x[t * H + h]);
+      } else {
+        for (int64_t h = 0; h < H; ++h) xf[h] = (float)bf16_val(x[t * H + h]);
+        quantize_blocks(H, xf, xq, xs);
+        for (int64_t h = 0; h < H; ++h) a[h] = orc_e4m3_value(xq[h]) * (double)xs[h / 128];
+      }
+      if (g < sh->E) expert_row(sh, w, 0, g, a, hbuf, hf, hq, hs, y_out + i * H);
+      else expert_row(sh, w, 1, 0, a, hbuf, hf, hq, hs, y_out + i * H);
+    }
+    free(a); free(hbuf); free(hf); free(hq); free(hs); free(xf); free(xq); free(xs);
+  }
 }

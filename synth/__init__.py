@@ -18,6 +18,9 @@ Recipe (all seeded; the values never depend on thread count):
   shared sw1, sw3, sw2: same laws, E = 1, their own tensor ids
   FP8 storage: the same bf16 draws quantised per 128x128 block,
                scale = blockmax/448 (fp32), codes E4M3 round-to-nearest-even.
+  NVFP4 storage: the same bf16 draws; per matrix a global fp32 scale
+               amax/(6*448); per 16 inputs an E4M3 scale of blockmax/(6*global);
+               E2M1 codes (nearest, ties to even, saturating), two to a byte.
   Skewed routing: router_bias[e] = -1.1 * alpha * ln(r_e), r a seeded random
                permutation of 1..E (Zipf exponent 1.1 over a random expert
                ranking); alpha = 0.25 makes the hottest expert take about ten
@@ -46,7 +49,7 @@ ID_SW1, ID_SW3, ID_SW2 = 20, 21, 22
 ZIPF_S = 1.1
 ZIPF_ALPHA = 0.25
 
-WDTYPE_BF16, WDTYPE_FP8 = 0, 1
+WDTYPE_BF16, WDTYPE_FP8, WDTYPE_NVFP4 = 0, 1, 2
 
 
 def build(force: bool = False) -> str:
@@ -69,6 +72,9 @@ def _load():
         lib.synth_fp8_blocks.argtypes = [u64, u64, i64, i64, i64, dbl, vp, vp]
         lib.synth_e4m3_value.argtypes = [ctypes.c_uint8]
         lib.synth_e4m3_value.restype = ctypes.c_float
+        lib.synth_e2m1_value.argtypes = [ctypes.c_uint8]
+        lib.synth_e2m1_value.restype = ctypes.c_float
+        lib.synth_nvfp4.argtypes = [u64, u64, i64, i64, i64, dbl, vp, vp, vp]
         _lib = lib
     return _lib
 
@@ -107,6 +113,26 @@ def fp8_blocks(seed: int, tid: int, G: int, rows: int, cols: int, std: float):
     scales = np.empty((G, rows // 128, cols // 128), dtype=np.float32)
     _load().synth_fp8_blocks(seed, tid, G, rows, cols, float(std), _ptr(codes), _ptr(scales))
     return codes, scales
+
+
+def nvfp4(seed: int, tid: int, G: int, rows: int, cols: int, std: float):
+    """NVFP4 version of normal_bf16(seed, tid, (G, rows, cols), std).
+
+    Returns (codes uint8 [G, rows, cols/2], E4M3 scales uint8 [G, rows, cols/16],
+    global scales fp32 [G]).
+    """
+    assert cols % 16 == 0
+    codes = np.empty((G, rows, cols // 2), dtype=np.uint8)
+    scales = np.empty((G, rows, cols // 16), dtype=np.uint8)
+    gs = np.empty(G, dtype=np.float32)
+    _load().synth_nvfp4(seed, tid, G, rows, cols, float(std), _ptr(codes), _ptr(scales), _ptr(gs))
+    return codes, scales, gs
+
+
+def e2m1_value_table() -> np.ndarray:
+    """The generator's own decoding of all 16 E2M1 codes."""
+    lib = _load()
+    return np.array([lib.synth_e2m1_value(c) for c in range(16)], dtype=np.float32)
 
 
 def e4m3_value_table() -> np.ndarray:
@@ -172,8 +198,10 @@ def make_weights(shape: MoeShape) -> dict:
     """Router and expert weights for `shape` (numpy, host memory).
 
     BF16 storage: uint16 bf16 bit patterns. FP8 storage: uint8 E4M3 codes plus
-    fp32 block scales. Keys: router_w, router_bias (None unless skewed),
-    w1, w3, w2, s1, s3, s2, sw1, sw3, sw2, ss1, ss3, ss2.
+    fp32 block scales. NVFP4 storage: packed E2M1 codes, E4M3 scales per 16
+    inputs and fp32 global scales (g1, g3, g2, sg1, sg3, sg2). Keys: router_w,
+    router_bias (None unless skewed), w1, w3, w2, s1, s3, s2, sw1, sw3, sw2,
+    ss1, ss3, ss2, g1, g3, g2, sg1, sg3, sg2.
     """
     H, E, I, s = shape.hidden, shape.n_experts, shape.inter, shape.seed
     wt = {"router_w": normal_bf16(s, ID_ROUTER_W, (E, H), 1.0 / math.sqrt(H)),
@@ -184,11 +212,14 @@ def make_weights(shape: MoeShape) -> dict:
                   ("sw2", "ss2", ID_SW2, 1, H, I, I)]
     for wname, sname, tid, G, rows, cols, fan_in in specs:
         std = 1.0 / math.sqrt(fan_in)
+        gname = ("s" if wname.startswith("sw") else "") + "g" + wname[-1]
         if shape.wdtype == WDTYPE_FP8:
             wt[wname], wt[sname] = fp8_blocks(s, tid, G, rows, cols, std)
+        elif shape.wdtype == WDTYPE_NVFP4:
+            wt[wname], wt[sname], wt[gname] = nvfp4(s, tid, G, rows, cols, std)
         else:
             wt[wname], wt[sname] = normal_bf16(s, tid, (G, rows, cols), std), None
-    for k in ("sw1", "sw3", "sw2", "ss1", "ss3", "ss2"):
+    for k in ("sw1", "sw3", "sw2", "ss1", "ss3", "ss2", "g1", "g3", "g2", "sg1", "sg3", "sg2"):
         wt.setdefault(k, None)
     return wt
 

@@ -21,10 +21,13 @@
  * code = E4M3(value / scale) rounded to nearest even, saturating at 448; an
  * all-zero block gets scale 1 and zero codes. This is checkpoint preparation,
  * not part of the layer; it has its own E4M3 encoder (below), written apart
- * from the oracle's and the kernels'.
+ * from the oracle's and the kernels'. NVFP4 weights (E2M1 codes, an E4M3 scale
+ * per 16 inputs, an fp32 global scale) are prepared the same way, with this
+ * module's own E2M1 encoder.
  */
 #include <math.h>
 #include <stdint.h>
+#include <stdlib.h>
 #include <string.h>
 
 #define GOLDEN 0x9E3779B97F4A7C15ull
@@ -176,3 +179,71 @@ void synth_fp8_blocks(uint64_t seed, uint64_t id, int64_t G, int64_t rows, int64
 
 /* Decoded value of a code under this module's decoder (for input checks). */
 float synth_e4m3_value(uint8_t c) { return e4m3_decode_prep(c); }
+
+/* E2M1 (OCP 4-bit float: 1 sign, 2 exponent bits with bias 1, 1 mantissa bit;
+ * magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6) encoder: nearest magnitude, an exact
+ * tie to the even code, saturation at 6. This module's own, for checkpoint
+ * preparation. */
+static const float E2M1_MAG[8] = {0.0f, 0.5f, 1.0f, 1.5f, 2.0f, 3.0f, 4.0f, 6.0f};
+
+static inline uint8_t e2m1_encode_prep(float v) {
+  const uint8_t sign = (v < 0.0f || (v == 0.0f && signbit(v))) ? 8 : 0;
+  const float a = fabsf(v);
+  if (a >= 6.0f) return sign | 7;
+  int lo = 0;
+  while (lo < 7 && E2M1_MAG[lo + 1] <= a) ++lo; /* E2M1_MAG[lo] <= a < E2M1_MAG[lo + 1] */
+  const float dlo = a - E2M1_MAG[lo], dhi = E2M1_MAG[lo + 1] - a;
+  int c = (dlo < dhi) ? lo : (dhi < dlo ? lo + 1 : ((lo & 1) ? lo + 1 : lo));
+  return sign | (uint8_t)c;
+}
+
+float synth_e2m1_value(uint8_t c) { return (c & 8) ? -E2M1_MAG[c & 7] : E2M1_MAG[c & 7]; }
+
+/*
+ * NVFP4 weights for G stacked matrices of shape [rows, cols] (nn.Linear order,
+ * cols a multiple of 16), the way an NVFP4 checkpoint stores them: per matrix a
+ * global fp32 scale gs = amax / (6 * 448) (1 for an all-zero matrix); per 16
+ * consecutive inputs of a row an E4M3 scale s = E4M3(blockmax / (6 gs)); codes
+ * E2M1(v / (s gs)), two per byte with input 2j in the low nibble of byte j (all
+ * zero where s decodes to 0). Values are the bf16 draws of
+ * synth_normal_bf16(seed, id, G*rows*cols, std).
+ * codes [G, rows, cols/2] uint8; scales [G, rows, cols/16] uint8; gscale [G] fp32.
+ */
+void synth_nvfp4(uint64_t seed, uint64_t id, int64_t G, int64_t rows, int64_t cols, double std, uint8_t* codes,
+                 uint8_t* scales, float* gscale) {
+  const uint64_t key = tensor_key(seed, id);
+  const int64_t n = rows * cols;
+#pragma omp parallel
+  {
+    float* vals = (float*)malloc(sizeof(float) * (size_t)n);
+#pragma omp for schedule(dynamic, 1)
+    for (int64_t g = 0; g < G; ++g) {
+      float amax = 0.0f;
+      for (int64_t i = 0; i < n; i += 2) {
+        double z0, z1;
+        normal_pair(key, (uint64_t)((g * n + i) >> 1), &z0, &z1);
+        vals[i] = bf16_to_f32(f32_to_bf16_rne((float)(z0 * std)));
+        vals[i + 1] = bf16_to_f32(f32_to_bf16_rne((float)(z1 * std)));
+        if (fabsf(vals[i]) > amax) amax = fabsf(vals[i]);
+        if (fabsf(vals[i + 1]) > amax) amax = fabsf(vals[i + 1]);
+      }
+      const float gs = amax > 0.0f ? amax / (6.0f * 448.0f) : 1.0f;
+      gscale[g] = gs;
+      for (int64_t b = 0; b < n / 16; ++b) {
+        const float* v = vals + b * 16;
+        float bmax = 0.0f;
+        for (int i = 0; i < 16; ++i) if (fabsf(v[i]) > bmax) bmax = fabsf(v[i]);
+        const uint8_t sc = e4m3_encode_prep(bmax / (6.0f * gs));
+        const float s = e4m3_decode_prep(sc);
+        scales[g * (n / 16) + b] = sc;
+        uint8_t* dst = codes + g * (n / 2) + b * 8;
+        for (int i = 0; i < 16; i += 2) {
+          const uint8_t lo = s > 0.0f ? e2m1_encode_prep(v[i] / (s * gs)) : 0;
+          const uint8_t hi = s > 0.0f ? e2m1_encode_prep(v[i + 1] / (s * gs)) : 0;
+          dst[i / 2] = (uint8_t)(lo | (hi << 4));
+        }
+      }
+    }
+    free(vals);
+  }
+}

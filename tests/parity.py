@@ -8,7 +8,8 @@ k experts whose logits are all within MARGIN of the k-th largest are a correct
 answer, and the check is that the GPU's set is such a set.
 
 Outputs: relative Frobenius error ||out - ref|| / ||ref|| against the oracle's
-fp64 result, at most 1e-2 for BF16 experts and 2e-2 for FP8 experts.
+fp64 result, at most 1e-2 for BF16 experts and 2e-2 for FP8 experts, both
+pooled over the compared tokens and for every token (or expert row) on its own.
 """
 import numpy as np
 
@@ -62,6 +63,13 @@ def frob_rel(out: np.ndarray, ref: np.ndarray) -> float:
     out = out.astype(np.float64)
     ref = ref.astype(np.float64)
     return float(np.linalg.norm(out - ref) / max(np.linalg.norm(ref), 1e-300))
+
+
+def rows_rel(out: np.ndarray, ref: np.ndarray) -> np.ndarray:
+    """Relative Frobenius error of each row (last axis) on its own."""
+    out = out.astype(np.float64).reshape(-1, out.shape[-1])
+    ref = ref.astype(np.float64).reshape(-1, ref.shape[-1])
+    return np.linalg.norm(out - ref, axis=1) / np.maximum(np.linalg.norm(ref, axis=1), 1e-300)
 
 
 def bf16_bits_to_f64(a: np.ndarray) -> np.ndarray:

@@ -105,6 +105,73 @@ def test_residual_stream_argument_errors_need_no_device(lib):
     assert lib.moe_combine_residual(ctypes.byref(cfg), 0, None, None, None, None, None) == m.MOE_OK
 
 
+def test_grouped_gemm_and_hooks_argument_errors_need_no_device(lib):
+    cfg = m.make_config(256, 16, 2, 1, 128, m.MOE_WDTYPE_FP8_E4M3)
+    fake = {k: 1 << 20 for k in m.WEIGHT_FIELDS}
+    w = m.moe_weights(*[fake[k] for k in m.WEIGHT_FIELDS])
+    g = lib.moe_grouped_gemm
+    # moe_grouped_gemm(cfg, stage, R, offsets, a, a_scale, w, row_gate, out, out_scale, ws, ws_bytes, stream)
+    assert g(ctypes.byref(cfg), 0, 4, 1024, 2048, 4096, ctypes.byref(w), None, 8192, 8192, 16384, 1 << 20, None) == \
+        m.MOE_ERR_INVALID_ARG                                                              # bad stage
+    assert g(ctypes.byref(cfg), m.MOE_STAGE_DOWN, -1, 1024, 2048, 4096, ctypes.byref(w), None, 8192, None, 16384,
+             1 << 20, None) == m.MOE_ERR_INVALID_ARG                                       # negative R
+    assert g(ctypes.byref(cfg), m.MOE_STAGE_DOWN, 4, 1024, 2048, None, ctypes.byref(w), None, 8192, None, 16384,
+             1 << 20, None) == m.MOE_ERR_INVALID_ARG                                       # FP8 without scales
+    assert g(ctypes.byref(cfg), m.MOE_STAGE_GATE_UP, 4, 1024, 2048, 4096, ctypes.byref(w), None, 8192, None,
+             16384, 1 << 20, None) == m.MOE_ERR_INVALID_ARG                                # FP8 h without out_scale
+    assert g(ctypes.byref(cfg), m.MOE_STAGE_DOWN, 4, 1024, 2056, 4096, ctypes.byref(w), None, 8192, None, 16384,
+             1 << 20, None) == m.MOE_ERR_MISALIGNED                                        # A not 16-byte aligned
+    assert g(ctypes.byref(cfg), m.MOE_STAGE_DOWN, 4, 1024, 2048, 4096, ctypes.byref(w), None, 8192, None, 16384,
+             16, None) == m.MOE_ERR_WORKSPACE_TOO_SMALL
+    assert g(ctypes.byref(cfg), m.MOE_STAGE_DOWN, 0, 1024, 2048, 4096, ctypes.byref(w), None, 8192, None, 16384,
+             1 << 20, None) == m.MOE_OK                                                    # R = 0: no-op
+    assert lib.moe_debug_inject(7, 0) == m.MOE_ERR_INVALID_ARG
+    assert lib.moe_debug_inject(m.MOE_INJECT_NONE, 0) == m.MOE_OK
+
+
+def test_expert_parallel_argument_errors_need_no_device(lib):
+    arr = (ctypes.c_void_p * 17)(*([1 << 20] * 17))
+    r = lib.moe_ep_reduce
+    # moe_ep_reduce(n_ranks, partials, T, hidden, t0, t1, out, stream)
+    assert r(0, arr, 8, 256, 0, 8, 4096, None) == m.MOE_ERR_INVALID_ARG
+    assert r(17, arr, 8, 256, 0, 8, 4096, None) == m.MOE_ERR_UNSUPPORTED_SHAPE
+    assert r(2, arr, 8, 100, 0, 8, 4096, None) == m.MOE_ERR_INVALID_ARG
+    assert r(2, arr, 8, 256, 4, 9, 4096, None) == m.MOE_ERR_INVALID_ARG
+    assert r(2, arr, 8, 256, 0, 8, 4100, None) == m.MOE_ERR_MISALIGNED
+    assert r(2, arr, 8, 256, 3, 3, 4096, None) == m.MOE_OK  # empty range: no launch
+    cfg = m.make_config(256, 16, 2, 1, 128, 0)
+    fake = {k: 1 << 20 for k in m.WEIGHT_FIELDS}
+    w = m.moe_weights(*[fake[k] for k in m.WEIGHT_FIELDS])
+    f = lib.moe_forward_ep_partial
+    # moe_forward_ep_partial(cfg, T, x, w, e0, e1, t0, t1, partial, idx, gate, ws, ws_bytes, stream)
+    assert f(ctypes.byref(cfg), 8, 4096, ctypes.byref(w), 4, 4, 0, 8, 8192, None, None, 16384, 1 << 30, None) == \
+        m.MOE_ERR_INVALID_ARG
+    assert f(ctypes.byref(cfg), 8, 4096, ctypes.byref(w), 0, 4, 0, 9, 8192, None, None, 16384, 1 << 30, None) == \
+        m.MOE_ERR_INVALID_ARG
+    assert f(ctypes.byref(cfg), 8, 4096, ctypes.byref(w), 0, 4, 0, 8, 8196, None, None, 16384, 1 << 30, None) == \
+        m.MOE_ERR_MISALIGNED
+    assert f(ctypes.byref(cfg), 0, 4096, ctypes.byref(w), 0, 4, 0, 0, 8192, None, None, 16384, 1 << 30, None) == \
+        m.MOE_OK
+
+
+def test_nvfp4_config_and_weight_checks_need_no_device(lib):
+    n = ctypes.c_size_t(0)
+    ok = m.make_config(4096, 352, 8, 1, 1536, m.MOE_WDTYPE_NVFP4)
+    assert lib.moe_workspace_bytes(ctypes.byref(ok), 64, ctypes.byref(n)) == m.MOE_OK
+    odd = m.make_config(384, 16, 2, 1, 256, m.MOE_WDTYPE_NVFP4)   # H not a multiple of 256
+    assert lib.moe_workspace_bytes(ctypes.byref(odd), 64, ctypes.byref(n)) == m.MOE_ERR_UNSUPPORTED_SHAPE
+    cfg = m.make_config(256, 16, 2, 1, 256, m.MOE_WDTYPE_NVFP4)
+    fake = {k: 1 << 20 for k in m.WEIGHT_FIELDS}
+    fake["router_bias"] = None
+    for missing in ("s2", "g1", "sg2"):
+        w = m.moe_weights(*[None if k == missing else fake[k] for k in m.WEIGHT_FIELDS])
+        assert lib.moe_forward(ctypes.byref(cfg), 4, 1024, ctypes.byref(w), 2048, None, None, 4096, 1 << 30,
+                               None) == m.MOE_ERR_INVALID_ARG, missing
+    w = m.moe_weights(*[(fake[k] + 8 if k == "s1" else fake[k]) for k in m.WEIGHT_FIELDS])
+    assert lib.moe_forward(ctypes.byref(cfg), 4, 1024, ctypes.byref(w), 2048, None, None, 4096, 1 << 30, None) == \
+        m.MOE_ERR_MISALIGNED
+
+
 def test_status_strings(lib):
     for c in range(8):
         assert m.moe_status_string(c) not in ("", "unknown status")

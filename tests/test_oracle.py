@@ -238,9 +238,24 @@ def _deq(codes_or_bits, scales, wdtype):
     return v * s
 
 
+# E2M1 magnitudes by code (OCP MX 4-bit float, written out: codes 0-7 are
+# 0, 0.5, 1, 1.5, 2, 3, 4, 6; bit 3 is the sign).
+E2M1_CLOSED_FORM = [0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0]
+
+
+def _deq_nvfp4(codes, scales, gs):
+    """[G, R, C] float64 from NVFP4 storage, by the closed-form E2M1 table and
+    torch's E4M3 decode (independent of the oracle's decoders)."""
+    mag = np.array(E2M1_CLOSED_FORM + [-v for v in E2M1_CLOSED_FORM])
+    lo, hi = mag[codes & 15], mag[codes >> 4]
+    v = np.stack([lo, hi], axis=-1).reshape(codes.shape[0], codes.shape[1], -1)
+    sc = torch.from_numpy(scales).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    return torch.from_numpy(v * np.repeat(sc, 16, axis=2) * gs.astype(np.float64)[:, None, None])
+
+
 def _act(x, wdtype):
     xf = torch.from_numpy(synth.bf16_to_f32(x).astype(np.float64))
-    if wdtype == synth.WDTYPE_BF16:
+    if wdtype in (synth.WDTYPE_BF16, synth.WDTYPE_NVFP4):
         return xf
     xr = xf.to(torch.float32).reshape(x.shape[0], -1, 128)
     amax = xr.abs().amax(dim=2, keepdim=True)
@@ -283,6 +298,89 @@ def test_layer_equals_brute_force_over_all_experts(wdtype):
     # the bf16 output is the fp64 sum rounded once
     assert np.array_equal(r["out_bf16"], torch.from_numpy(r["out_f64"]).to(torch.bfloat16).view(torch.int16)
                           .numpy().view(np.uint16))
+
+
+@pytest.mark.parametrize("wdtype", [synth.WDTYPE_BF16, synth.WDTYPE_FP8])
+def test_expert_rows_equal_dense_swiglu_per_expert(wdtype):
+    """Single (token, expert) rows, any expert (routed or not, and the shared
+    one), against torch's dense SwiGLU of that expert, and against moe_tokens."""
+    shape = synth.MoeShape("rows", T=12, hidden=256, n_experts=6, top_k=2, n_shared=1, inter=256,
+                           wdtype=wdtype, seed=23)
+    w = synth.make_weights(shape)
+    x = synth.make_x(shape)
+    toks = np.repeat(np.arange(shape.T), shape.n_experts + 1)
+    grps = np.tile(np.arange(shape.n_experts + 1), shape.T)
+    y = oracle.expert_rows(shape, w, x, toks, grps).reshape(shape.T, shape.n_experts + 1, -1)
+    a = _act(x, wdtype)
+    W1, W3, W2 = (_deq(w[p], w[q], wdtype) for p, q in (("w1", "s1"), ("w3", "s3"), ("w2", "s2")))
+    SW1, SW3, SW2 = (_deq(w[p], w[q], wdtype)[0] for p, q in (("sw1", "ss1"), ("sw3", "ss3"), ("sw2", "ss2")))
+    for e in range(shape.n_experts + 1):
+        ref = (_dense_swiglu_torch(a, W1[e], W3[e], W2[e], wdtype) if e < shape.n_experts
+               else _dense_swiglu_torch(a, SW1, SW3, SW2, wdtype)).numpy()
+        err = np.linalg.norm(y[:, e] - ref) / np.linalg.norm(ref)
+        assert err < 1e-6, (e, err)
+    idx, gate, _ = oracle.route(x, w["router_w"], None, shape.top_k)
+    _, _, ys = oracle.moe_tokens(shape, w, x, idx, gate, want_y=True)
+    for t in range(shape.T):
+        for j in range(shape.top_k):
+            assert np.array_equal(ys[t, j], y[t, idx[t, j]])
+        assert np.array_equal(ys[t, shape.top_k], y[t, shape.n_experts])
+
+
+def test_e2m1_decode_every_code():
+    got = oracle.e2m1_decode(np.arange(16, dtype=np.uint8))
+    want = np.array(E2M1_CLOSED_FORM + [-v for v in E2M1_CLOSED_FORM])
+    assert np.array_equal(got, want)
+    assert np.all(np.signbit(got[8:]))                       # code 8 is -0
+    assert np.array_equal(got, synth.e2m1_value_table().astype(np.float64))  # the generator's own decoder
+
+
+def test_nvfp4_nibble_order_and_scales():
+    # one row of 32 inputs: bytes j hold inputs 2j (low nibble) and 2j+1 (high)
+    codes = np.zeros((1, 16), np.uint8)
+    codes[0, 0] = 0x7A          # input 0: code 0xA = -1, input 1: code 7 = 6
+    codes[0, 9] = 0x21          # input 18: code 1 = 0.5, input 19: code 2 = 1
+    scales = np.array([[0x38, 0x40]], np.uint8)  # E4M3 1.0 for inputs 0-15, 2.0 for 16-31
+    w = oracle.nvfp4_dequantize(codes, scales, 0.25)
+    want = np.zeros(32)
+    want[0], want[1], want[18], want[19] = -0.25, 1.5, 0.25, 0.5
+    assert np.array_equal(w[0], want)
+
+
+def test_nvfp4_generator_keeps_values_within_the_format_error():
+    """The checkpoint preparation (input side): dequantised NVFP4 weights stay
+    within half an E2M1 step (times the block scale) of the bf16 draws."""
+    G, R, C, std = 2, 64, 256, 0.05
+    codes, scales, gs = synth.nvfp4(3, 99, G, R, C, std)
+    ref = synth.bf16_to_f32(synth.normal_bf16(3, 99, (G, R, C), std)).astype(np.float64)
+    deq = _deq_nvfp4(codes, scales, gs).numpy()
+    assert np.allclose(gs, np.abs(ref).reshape(G, -1).max(axis=1) / (6 * 448), rtol=1e-6)
+    step = np.repeat(torch.from_numpy(scales).view(torch.float8_e4m3fn).to(torch.float64).numpy(), 16, axis=2) \
+        * gs[:, None, None]
+    assert np.all(np.abs(deq - ref) <= step * 1.0 + 1e-12)   # the widest E2M1 gap is 2 (4 -> 6)
+    assert np.linalg.norm(deq - ref) / np.linalg.norm(ref) < 0.15
+
+
+def test_nvfp4_layer_equals_brute_force_over_all_experts():
+    shape = synth.MoeShape("bf-nvfp4", T=16, hidden=256, n_experts=6, top_k=2, n_shared=1, inter=256,
+                           wdtype=synth.WDTYPE_NVFP4, seed=24)
+    w = synth.make_weights(shape)
+    x = synth.make_x(shape)
+    r = oracle.moe_forward(shape, w, x)
+    a = _act(x, shape.wdtype)
+    W1, W3, W2 = (_deq_nvfp4(w[p], w[q], w[g]) for p, q, g in (("w1", "s1", "g1"), ("w3", "s3", "g3"),
+                                                                ("w2", "s2", "g2")))
+    SW1, SW3, SW2 = (_deq_nvfp4(w[p], w[q], w[g])[0] for p, q, g in (("sw1", "ss1", "sg1"), ("sw3", "ss3", "sg3"),
+                                                                       ("sw2", "ss2", "sg2")))
+    bf = synth.WDTYPE_BF16  # NVFP4 keeps bf16 activations and rounds h to bf16
+    Y = torch.stack([_dense_swiglu_torch(a, W1[e], W3[e], W2[e], bf) for e in range(shape.n_experts)])
+    G = torch.zeros(shape.T, shape.n_experts, dtype=torch.float64)
+    for t in range(shape.T):
+        for j in range(shape.top_k):
+            G[t, r["idx"][t, j]] = float(r["gate"][t, j])
+    ref = torch.einsum("te,eth->th", G, Y) + _dense_swiglu_torch(a, SW1, SW3, SW2, bf)
+    err = np.linalg.norm(r["out_f64"] - ref.numpy()) / np.linalg.norm(ref.numpy())
+    assert err < 1e-6, err
 
 
 def test_token_subset_equals_full_run():

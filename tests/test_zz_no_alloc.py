@@ -51,6 +51,53 @@ def test_noalloc_permute_matches_moe_permute_on_two_calls():
             assert torch.equal(a, b), f"call {call}: {name} differs"
 
 
+@pytest.mark.parametrize("T", [1, 64, 256, 257])
+def test_noalloc_permute_matches_the_one_chunk_path(T):
+    """T <= 256: moe_permute takes its one-launch path, this entry point the
+    three-kernel one; both must give the same rows."""
+    import torch
+    import mixture_experts_histogram_b200 as m
+    E, k, S = 352, 8, 1
+    G = E + S
+    cfg = m.make_config(4096, E, k, S, 1536, 1)
+    idx = m.to_device(_routing(T, E, k, 40 + T))
+    ref = [torch.empty(G, dtype=torch.int32, device="cuda"), torch.empty(G + 1, dtype=torch.int32, device="cuda"),
+           torch.empty((k + S) * T, dtype=torch.int32, device="cuda"),
+           torch.empty((T, k + S), dtype=torch.int32, device="cuda")]
+    ws = torch.empty(m.moe_workspace_bytes(cfg, T), dtype=torch.uint8, device="cuda")
+    m.moe_permute(cfg, T, idx, *ref, ws)
+    got = [torch.full_like(t, -7) for t in ref]
+    status = torch.full((1,), 99, dtype=torch.int32, device="cuda")
+    m.moe_permute_noalloc(cfg, T, idx, *got, device_status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    for name, a, b in zip(("counts", "offsets", "perm", "pos"), ref, got):
+        assert torch.equal(a, b), f"T={T}: {name} differs"
+
+
+def test_noalloc_permute_zero_tokens_and_bad_index():
+    import torch
+    import mixture_experts_histogram_b200 as m
+    E, k, S = 16, 2, 1
+    cfg = m.make_config(256, E, k, S, 128, 0)
+    counts = torch.full((E + S,), 5, dtype=torch.int32, device="cuda")
+    offsets = torch.full((E + S + 1,), 5, dtype=torch.int32, device="cuda")
+    status = torch.full((1,), 99, dtype=torch.int32, device="cuda")
+    m.moe_permute_noalloc(cfg, 0, 1024, counts, offsets, 1024, 1024, device_status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    assert torch.count_nonzero(counts).item() == 0 and torch.count_nonzero(offsets).item() == 0
+    T = 300
+    idx_np = np.tile(np.array([[0, 1]], np.int32), (T, 1))
+    idx_np[5, 1] = 99
+    perm = torch.empty((k + S) * T, dtype=torch.int32, device="cuda")
+    pos = torch.empty((T, k + S), dtype=torch.int32, device="cuda")
+    m.moe_permute_noalloc(cfg, T, m.to_device(idx_np), counts, offsets, perm, pos, device_status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == m.MOE_ERR_BAD_INDEX
+    assert pos[5, 1].item() == -1 and counts[1].item() == T - 1
+
+
 def test_noalloc_permute_refuses_sizes_beyond_its_scratch():
     import mixture_experts_histogram_b200 as m
     cfg = m.make_config(4096, 352, 8, 1, 1536, 1)
