@@ -42,7 +42,8 @@ def parse_args():
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=["prefill-fp8", "decode-bf16", "long-skew-fp8", "dense-ffn-fp8"],
+    ap.add_argument("--workload", choices=["prefill-fp8", "decode-bf16", "long-skew-fp8", "dense-ffn-fp8",
+                                           "nvfp4"],
                     default="prefill-fp8")
     ap.add_argument("--no-decode", action="store_true", help="skip the T=64 FP8 decode line")
     ap.add_argument("--no-extra", action="store_true",
@@ -60,7 +61,7 @@ def workload(name, tokens=None, experts=None):
     import dataclasses
     import synth
     s = {"prefill-fp8": synth.PREFILL_FP8, "decode-bf16": synth.DECODE_BF16,
-         "long-skew-fp8": synth.LONG_SKEW_FP8, "dense-ffn-fp8": synth.DENSE_FFN_FP8}[name]
+         "long-skew-fp8": synth.LONG_SKEW_FP8, "dense-ffn-fp8": synth.DENSE_FFN_FP8, "nvfp4": synth.STEP5_NVFP4}[name]
     if experts is not None:
         s = dataclasses.replace(s, n_experts=experts, name=f"{s.name}-E{experts}")
     if tokens is not None:
@@ -68,10 +69,14 @@ def workload(name, tokens=None, experts=None):
     return s
 
 
+STORAGE = {0: "BF16", 1: "FP8 E4M3 128x128 weights, 1x128 activations",
+           2: "NVFP4 weights (E2M1, E4M3 per 16, fp32 global), bf16 activations"}
+
+
 def describe(shape) -> dict:
     return {"workload": f"{shape.name}: T={shape.T} H={shape.hidden} E={shape.n_experts} top-{shape.top_k} "
                         f"shared={shape.n_shared} I={shape.inter} "
-                        f"{'FP8 E4M3 128x128 weights, 1x128 activations' if shape.wdtype else 'BF16'}"
+                        f"{STORAGE[shape.wdtype]}"
                         f"{', Zipf-skewed routing' if shape.skew else ', uniform routing'}",
             "tokens": shape.T, "hidden": shape.hidden, "experts": shape.n_experts, "top_k": shape.top_k,
             "shared_experts": shape.n_shared, "inter": shape.inter, "seed": shape.seed,
@@ -326,7 +331,8 @@ def run_ours(args):
         # The long skewed prefill and the FP8 decode sweep, each on its own
         # seeded weights (freed between workloads).
         for key, wshape, tokens in (("long_skew_t32768", synth.LONG_SKEW_FP8, [synth.LONG_SKEW_FP8.T]),
-                                    ("decode_sweep_fp8", synth.SWEEP_FP8, list(synth.SWEEP_TOKENS))):
+                                    ("decode_sweep_fp8", synth.SWEEP_FP8, list(synth.SWEEP_TOKENS)),
+                                    ("nvfp4_w4a16", synth.STEP5_NVFP4, [64, 8192])):
             wd = wts = None
             torch.cuda.empty_cache()
             ew = m.upload_weights(synth.make_weights(wshape), f"cuda:{local}")
@@ -342,17 +348,25 @@ def run_ours(args):
         """The dominant kernel against its bound (HBM bytes or tensor FLOPs)."""
         idx = res["idx"]
         touched = int(np.unique(idx).size)
-        es = 1 if shape.wdtype else 2
+        fp8 = shape.wdtype == synth.WDTYPE_FP8
+        es = 1 if fp8 else 2  # activation bytes (x, h); NVFP4 keeps bf16 activations
         H, I, E, k, S = shape.hidden, shape.inter, shape.n_experts, shape.top_k, shape.n_shared
         R = (k + S) * T
         groups = touched + S
-        scale1 = (2 * (I // 128) * (H // 128) * 4) if shape.wdtype else 0
-        scale2 = ((H // 128) * (I // 128) * 4) if shape.wdtype else 0
+
+        def wbytes(rows, cols):
+            """Stored bytes of one expert matrix [rows, cols], scales included."""
+            if fp8:
+                return rows * cols + (rows // 128) * (cols // 128) * 4
+            if shape.wdtype == synth.WDTYPE_NVFP4:
+                return rows * cols // 2 + rows * cols // 16 + 4
+            return rows * cols * 2
+
         kern = {
             "gemm1_gate_up_swiglu": {
-                "bytes": groups * (2 * I * H * es + scale1) + T * H * es + R * I * es,
+                "bytes": groups * 2 * wbytes(I, H) + T * H * es + R * I * es,
                 "flops": 2.0 * R * H * 2 * I},
-            "gemm2_down": {"bytes": groups * (H * I * es + scale2) + R * I * es + R * H * 2,
+            "gemm2_down": {"bytes": groups * wbytes(H, I) + R * I * es + R * H * 2,
                            "flops": 2.0 * R * I * H},
         }
         for kk, v in kern.items():
@@ -362,11 +376,11 @@ def run_ours(args):
                 v["hbm_gbs"] = round(v["bytes"] / (kms / 1e3) / 1e9, 1)
                 v["hbm_frac"] = round(v["hbm_gbs"] / pk["hbm_gbs"], 4)
                 v["tflops"] = round(v["flops"] / (kms / 1e3) / 1e12, 1)
-                v["tensor_frac"] = round(v["tflops"] / (pk["fp8_tflops"] if shape.wdtype else pk["bf16_tflops"]), 4)
+                v["tensor_frac"] = round(v["tflops"] / (pk["fp8_tflops"] if fp8 else pk["bf16_tflops"]), 4)
         dom = max(kern, key=lambda kk: res["kernel_ms"].get(kk, 0.0))
         ms = res["kernel_ms"][dom]
         t_hbm = kern[dom]["bytes"] / (pk["hbm_gbs"] * 1e9)
-        peak_tf = pk["fp8_tflops"] if shape.wdtype else pk["bf16_tflops"]
+        peak_tf = pk["fp8_tflops"] if fp8 else pk["bf16_tflops"]  # NVFP4 runs bf16 MMAs
         t_tc = kern[dom]["flops"] / (peak_tf * 1e12)
         traffic = traffic_for(dom, shape.name if T == shape.T else f"{shape.name}@T={T}")
         if t_hbm >= t_tc:
@@ -380,7 +394,7 @@ def run_ours(args):
                   "algorithmic_flops": kern[dom]["flops"], "touched_experts": touched,
                   "peak_source": f"{pk['source']} (MEASURED_PEAKS.json; FP8 = 2 x measured BF16)"})
         # Whole layer against max(compute, bytes): weights of touched experts + router + x + out.
-        lay_bytes = (groups * (3 * I * H * es + scale1 + scale2) + E * H * 2 + 2 * T * H * 2)
+        lay_bytes = groups * (2 * wbytes(I, H) + wbytes(H, I)) + E * H * 2 + 2 * T * H * 2
         lay_flops = 2.0 * T * H * E + 2.0 * 3 * H * I * R
         t_roof = max(lay_bytes / (pk["hbm_gbs"] * 1e9), lay_flops / (peak_tf * 1e12))
         layer = {"ms": round(res["ms_per_step"], 4), "roofline_ms": round(t_roof * 1e3, 4),
@@ -396,7 +410,8 @@ def run_ours(args):
         "metric": METRIC, "value": round(main["tokens_per_s"], 1), "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(main["ms_per_step"], 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "e4m3" if shape.wdtype else "bf16", "data": "synthetic (seeded, counter-based generator)",
+        "dtype": {0: "bf16", 1: "e4m3", 2: "nvfp4 weights, bf16 activations"}[shape.wdtype],
+        "data": "synthetic (seeded, counter-based generator)",
         "config": dict(describe(shape), parallelism=f"replicas x{world}" if world > 1 else "single GPU"),
         "roofline": roof, "layer_roofline": layer,
         "kernel_ms": {k: round(v, 4) for k, v in main["kernel_ms"].items()},

@@ -184,6 +184,19 @@ int run_route(const moe_config* c, const WsLayout& L, int64_t T, const void* x, 
   CUtensorMap tx, tw;
   if (!map_2d(&tx, x, false, c->hidden, T, 64, kTileM)) return MOE_ERR_CUDA;
   if (!map_2d(&tw, router_w, false, c->hidden, c->n_experts, 64, rp.box_rows)) return MOE_ERR_CUDA;
+  if (rp.ksplit == 1) {
+    // One CTA holds each token tile's whole K sum: the top-k runs in its epilogue.
+    rp.fused = 1;
+    rp.k = c->top_k;
+    rp.bias = bias;
+    rp.idx = idx;
+    rp.gate = gate;
+    rp.logits = logits;
+    CUDA_TRY(launch_router_gemm(rp, tx, tw, s));
+    prof.mark();
+    prof.mark();  // no separate top-k kernel
+    return MOE_OK;
+  }
   CUDA_TRY(launch_router_gemm(rp, tx, tw, s));
   prof.mark();
   TopkParams tp{};

@@ -40,8 +40,14 @@ struct RouterParams {
   int32_t box_rows;     // rows per B box (multiple of 16, <= 256)
   int32_t ksplit;       // K splits (grid.y)
   int32_t kstages;      // total K stages (H / 64)
-  float* partial;       // [ksplit, T, E] fp32
+  float* partial;       // [ksplit, T, E] fp32 (unfused)
   int* status;
+  // Fused top-k (ksplit == 1): the epilogue selects and writes idx/gate itself.
+  int32_t fused, k;
+  const float* bias;    // [E] or null
+  int32_t* idx;         // [T, k]
+  float* gate;          // [T, k]
+  float* logits;        // [T, E] or null
 };
 
 struct TopkParams {

@@ -12,7 +12,8 @@
 // thread, 32 columns at a time), transpose each 32 x 32 block through shared
 // memory and store fp32 partial logits as whole 128-byte row segments. Small T is split along K so that the
 // 2.9 MB of router weights are streamed by many SMs at once; the top-k kernel
-// adds the K-split partials in a fixed order.
+// adds the K-split partials in a fixed order. Without a K split (T >= 148 x 128
+// tokens) the selection is fused into this kernel's epilogue instead.
 #include <cuda_bf16.h>
 #include <math.h>
 
@@ -33,6 +34,65 @@ __host__ __device__ inline int router_stages(const RouterParams& p) {
   const int per = kASmem + router_b_bytes(p);
   int st = (200 * 1024) / per;
   return st > kRouterMaxStages ? kRouterMaxStages : st;
+}
+
+// The whole K sum of this thread's token row is in TMEM (no K split): the
+// token's logits (plus bias) stream through registers 32 columns at a time and
+// a sorted list of the kTop largest (the earlier, lower index wins a tie, as a
+// later equal value never displaces it) is kept by insertion; then the gates
+// are the chosen logits' softmax. Every lane of the warp takes part in the TMEM
+// loads; lanes past the last token only skip the writes.
+template <int kTop>
+__device__ __forceinline__ void fused_topk(const RouterParams& p, uint32_t taddr, int64_t t, int ncols, int lane) {
+  float top_v[kTop];
+  int top_e[kTop];
+#pragma unroll
+  for (int j = 0; j < kTop; ++j) {
+    top_v[j] = -INFINITY;
+    top_e[j] = 0x7fffffff;
+  }
+  const bool live = t < p.T;
+  for (int c0 = 0; c0 < ncols; c0 += 32) {
+    uint32_t v[32];
+    tmem_ld32(taddr + (uint32_t)c0, v);
+    tmem_ld_wait();
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      const int e = c0 + i;
+      if (e >= p.E) break;
+      float l = __uint_as_float(v[i]);
+      if (p.bias) l += __ldg(p.bias + e);
+      if (live && p.logits) p.logits[t * p.E + e] = l;
+      if (l > top_v[kTop - 1]) {
+        float cv = l;
+        int ce = e;
+#pragma unroll
+        for (int j = 0; j < kTop; ++j) {
+          const bool sw = cv > top_v[j];
+          const float tv = top_v[j];
+          const int te = top_e[j];
+          top_v[j] = sw ? cv : tv;
+          top_e[j] = sw ? ce : te;
+          cv = sw ? tv : cv;
+          ce = sw ? te : ce;
+        }
+      }
+    }
+  }
+  if (!live) return;
+  float w[kTop], z = 0.0f;
+#pragma unroll
+  for (int j = 0; j < kTop; ++j) {
+    w[j] = j < p.k ? expf(top_v[j] - top_v[0]) : 0.0f;
+    z += w[j];
+  }
+#pragma unroll
+  for (int j = 0; j < kTop; ++j) {
+    if (j < p.k) {
+      p.idx[t * p.k + j] = top_e[j];
+      p.gate[t * p.k + j] = w[j] / z;
+    }
+  }
 }
 
 __global__ void __launch_bounds__(kRouterThreads, 1)
@@ -121,7 +181,11 @@ __global__ void __launch_bounds__(kRouterThreads, 1)
     const int q = warp % 4;
     bool ok = mbar_wait(done, 0, p.status, abort_flag);
     ok = __all_sync(0xffffffffu, ok);
-    if (ok) {
+    if (ok && p.fused) {
+      tc_fence_after_sync();
+      if (p.k <= 8) fused_topk<8>(p, tmem + ((uint32_t)(q * 32) << 16), m_tile * kTileM + q * 32 + lane, ncols, lane);
+      else fused_topk<kMaxTopK>(p, tmem + ((uint32_t)(q * 32) << 16), m_tile * kTileM + q * 32 + lane, ncols, lane);
+    } else if (ok) {
       tc_fence_after_sync();
       // Every MMA has completed (done), so the stage buffers are free: each
       // warp transposes through its own 32 x 33 float block of them.

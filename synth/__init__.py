@@ -178,7 +178,12 @@ SWEEP_TOKENS = (1, 8, 64, 512, 2048)
 DENSE_FFN_FP8 = MoeShape("step5-dense-ffn-fp8", T=8192, n_experts=1, top_k=1, n_shared=0, inter=13824,
                          wdtype=WDTYPE_FP8, seed=5)
 
-WORKLOADS = {w.name: w for w in (TINY, DECODE_BF16, PREFILL_FP8, LONG_SKEW_FP8, SWEEP_FP8, DENSE_FFN_FP8)}
+# The Step-5 layer with NVFP4 expert storage (W4A16), the storage variant of
+# the TensorFold PR page, at the decode shape.
+STEP5_NVFP4 = MoeShape("step5-nvfp4-w4a16", T=64, wdtype=WDTYPE_NVFP4, seed=6)
+
+WORKLOADS = {w.name: w for w in (TINY, DECODE_BF16, PREFILL_FP8, LONG_SKEW_FP8, SWEEP_FP8, DENSE_FFN_FP8,
+                                 STEP5_NVFP4)}
 
 
 def zipf_bias(seed: int, E: int, alpha: float = ZIPF_ALPHA) -> np.ndarray:
