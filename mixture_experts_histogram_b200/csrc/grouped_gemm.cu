@@ -538,9 +538,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             acc[i].y = silu_mul(acc[i].y, acc[32 + i].y);
             amax = fmaxf(amax, fmaxf(fabsf(acc[i].x), fabsf(acc[i].y)));
           }
+          // The two warps that share this row quarter (same q, other column
+          // half) exchange their maxima; a 64-thread barrier per pair.
           float* ax = amax_x + (tile_iter & 1u) * 256;
           ax[hf * 128 + rl] = amax;
-          named_bar_sync(1, kEpiThreads);
+          named_bar_sync(1 + q, 64);
           amax = fmaxf(amax, ax[(1 - hf) * 128 + rl]);
           const float s = amax > 0.0f ? __fdiv_rn(amax, 448.0f) : 1.0f;
           const float inv = amax > 0.0f ? __frcp_rn(s) : 0.0f;

@@ -24,7 +24,7 @@
 //   warp 0       producer: TMA of the activation tile (into the MMA ring), of
 //                the weight codes (256 rows x 32 bytes per 64-deep K stage, into
 //                a raw ring) and, every 4 stages, of their scales (256 rows x 16
-//                bytes) into a two-slot scale ring.
+//                bytes) into a small scale ring.
 //   warp 1       TMEM allocation (512 columns) and the single-thread MMA issuer.
 //   warps 2-9    epilogue (two column halves x four TMEM lane quarters).
 //   warps 10-17  converters: codes x scales -> bf16 weight tile, then a proxy
@@ -43,8 +43,21 @@ namespace {
 constexpr int kConvWarps = 8;
 constexpr int kEpiWarpsNv = 8;
 constexpr int kNvThreads = 32 * (2 + kEpiWarpsNv + kConvWarps);
-constexpr int kConvStages = 3;                 // A + converted B tiles (the MMA's ring)
-constexpr int kRawStages = 4;                  // codes (the converters' ring); a scale slot spans 4 stages
+#ifndef MOE_NV_CONV_STAGES
+#define MOE_NV_CONV_STAGES 3
+#endif
+#ifndef MOE_NV_RAW_STAGES
+#define MOE_NV_RAW_STAGES 4
+#endif
+constexpr int kConvStages = MOE_NV_CONV_STAGES;  // A + converted B tiles (the MMA's ring)
+constexpr int kRawStages = MOE_NV_RAW_STAGES;    // codes (the converters' ring)
+// A scale slot serves 4 stages. The producer refills the slot of scale group
+// G at stage 4G after the converters finished stage 4G - kRawStages, so the
+// slot's previous group (G - kScaleSlots) must end by then:
+// 4 (G - kScaleSlots) + 3 <= 4G - kRawStages.
+constexpr int kScaleSlots = (kRawStages + 3 + 3) / 4;
+static_assert(4 * kScaleSlots >= kRawStages + 3, "scale slots too few for the raw ring");
+static_assert(kRawStages >= 4 && kRawStages <= 24 && kConvStages <= 8, "ring sizes fit the drain bitmask");
 constexpr int kABytesNv = kTileM * 128;        // 128 rows x 64 bf16
 constexpr int kBRows = 256;
 constexpr int kBBytesNv = kBRows * 128;        // 256 rows x 64 bf16
@@ -56,7 +69,7 @@ struct NvLayout {
   static constexpr size_t kB = kA + (size_t)kConvStages * kABytesNv;
   static constexpr size_t kCodes = kB + (size_t)kConvStages * kBBytesNv;
   static constexpr size_t kScales = kCodes + (size_t)kRawStages * kCodeBytes;
-  static constexpr size_t kBars = kScales + 2 * (size_t)kScaleSlotBytes;
+  static constexpr size_t kBars = kScales + (size_t)kScaleSlots * kScaleSlotBytes;
   static constexpr int kNumBars = 2 * kConvStages + 2 * kRawStages + 2 + 2 + 1;
   static constexpr size_t kMisc = kBars + ((kNumBars * 8 + 127) / 128) * 128;  // tmem slot, abort flag
   static constexpr size_t kMt = kMisc + 64;
@@ -166,7 +179,7 @@ __global__ void __launch_bounds__(kNvThreads, 1)
     // ------------------------------------------------------------ producer --
     if (lane == 0) {
       uint32_t it_raw = 0, it_conv = 0;
-      uint32_t issued = 0, issued_phase = 0;  // raw ring (bit s) and MMA ring (bit 8 + s)
+      uint32_t issued = 0, issued_phase = 0;  // raw ring (bit s) and MMA ring (bit 24 + s)
       bool ok = true;
       for (int item = blockIdx.x; item < total && ok && p.inject != 1; item += gridDim.x) {
         const Item it = decode_item(item, p.n_tiles, p.G, kTileM, s_mt, s_off, p.n_fastest != 0);
@@ -185,7 +198,7 @@ __global__ void __launch_bounds__(kNvThreads, 1)
           const uint32_t rs = it_raw % kRawStages, rph = (it_raw / kRawStages) & 1u;
           if (!mbar_wait(&rempty[rs], rph ^ 1u, p.status, abort_flag, site0 | 1, item, p.wait_ns)) { ok = false; break; }
           const bool with_scales = (ks & 3) == 0;
-          const uint32_t ss = (it_raw / 4) & 1u;
+          const uint32_t ss = (it_raw / 4) % kScaleSlots;
           mbar_arrive_expect_tx(&rfull[rs], kCodeBytes + (with_scales ? kScaleSlotBytes : 0));
           uint8_t* cdst = sCodes + rs * kCodeBytes;
           uint8_t* sdst = sScales + ss * kScaleSlotBytes;
@@ -207,16 +220,16 @@ __global__ void __launch_bounds__(kNvThreads, 1)
           if (!mbar_wait(&cempty[cs], cph ^ 1u, p.status, abort_flag, site0 | 2, item, p.wait_ns)) { ok = false; break; }
           mbar_arrive_expect_tx(&cfull[cs], (uint32_t)a_rows * 128u);
           tma_load_2d(sA + cs * kABytesNv, amap, &cfull[cs], ks * 64, it.row0);
-          issued |= 1u << (8 + cs);
-          issued_phase = (issued_phase & ~(1u << (8 + cs))) | (cph << (8 + cs));
+          issued |= 1u << (24 + cs);
+          issued_phase = (issued_phase & ~(1u << (24 + cs))) | (cph << (24 + cs));
           ++it_conv;
         }
       }
       if (!ok) {
         // Let the tensor copies already in flight land before the CTA leaves.
-        for (int s = 0; s < 8 + kConvStages; ++s) {
+        for (int s = 0; s < 24 + kConvStages; ++s) {
           if (!(issued & (1u << s))) continue;
-          uint64_t* bar = s < 8 ? &rfull[s] : &cfull[s - 8];
+          uint64_t* bar = s < 24 ? &rfull[s] : &cfull[s - 24];
           const uint64_t t0 = global_timer_ns();
           while (!mbar_try_wait(bar, (issued_phase >> s) & 1u) && global_timer_ns() - t0 < 200000000ull) {}
         }
@@ -353,7 +366,7 @@ __global__ void __launch_bounds__(kNvThreads, 1)
           break;
         }
         const uint8_t* codes = sCodes + rs * kCodeBytes;
-        const uint8_t* scl = sScales + ((it_raw / 4) & 1u) * kScaleSlotBytes + (ks & 3) * 4 + (c >> 1);
+        const uint8_t* scl = sScales + ((it_raw / 4) % kScaleSlots) * kScaleSlotBytes + (ks & 3) * 4 + (c >> 1);
         uint8_t* dst = sB + cs * kBBytesNv;
 #pragma unroll
         for (int i = 0; i < kBRows / 32; ++i) {
