@@ -368,13 +368,20 @@ __global__ void __launch_bounds__(kNvThreads, 1)
         const uint8_t* codes = sCodes + rs * kCodeBytes;
         const uint8_t* scl = sScales + ((it_raw / 4) % kScaleSlots) * kScaleSlotBytes + (ks & 3) * 4 + (c >> 1);
         uint8_t* dst = sB + cs * kBBytesNv;
+        // All loads first: the compiler cannot move a load from the code ring
+        // above a store into the weight tile (it cannot tell they never alias).
+        uint32_t w[kBRows / 32], sc[kBRows / 32];
 #pragma unroll
         for (int i = 0; i < kBRows / 32; ++i) {
           const int r = r0 + 32 * i;
-          const uint32_t w = *reinterpret_cast<const uint32_t*>(codes + r * 32 + c * 4);
-          const uint4 o = expand8(w, scl[r * 16]);
+          w[i] = *reinterpret_cast<const uint32_t*>(codes + r * 32 + c * 4);
+          sc[i] = scl[r * 16];
+        }
+#pragma unroll
+        for (int i = 0; i < kBRows / 32; ++i) {
+          const int r = r0 + 32 * i;
           // 128-byte swizzle: chunk c of row r lands at chunk c ^ (r % 8).
-          *reinterpret_cast<uint4*>(dst + r * 128 + ((c ^ (r & 7)) << 4)) = o;
+          *reinterpret_cast<uint4*>(dst + r * 128 + ((c ^ (r & 7)) << 4)) = expand8(w[i], sc[i]);
         }
         fence_proxy_async_smem();  // the MMA reads the tile through the async proxy
         __syncwarp();
