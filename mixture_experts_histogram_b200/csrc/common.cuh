@@ -127,6 +127,34 @@ struct CombineParams {
 // moe_launch_count) and returns `e`. Every launcher returns through it.
 cudaError_t counted_launch(cudaError_t e);
 
+// Launches `kern` on `s` with programmatic stream serialization (the kernel
+// calls pdl_wait() before its first global-memory access; see ptx.cuh) and, for
+// cluster_x > 1, clusters of cluster_x CTAs along x. Counted like every launch.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s, int cluster_x,
+                       Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[2];
+  int n = 0;
+  attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[n].val.programmaticStreamSerializationAllowed = 1;
+  ++n;
+  if (cluster_x > 1) {
+    attr[n].id = cudaLaunchAttributeClusterDimension;
+    attr[n].val.clusterDim.x = (unsigned)cluster_x;
+    attr[n].val.clusterDim.y = 1;
+    attr[n].val.clusterDim.z = 1;
+    ++n;
+  }
+  cfg.attrs = attr;
+  cfg.numAttrs = (unsigned)n;
+  return counted_launch(cudaLaunchKernelEx(&cfg, kern, static_cast<Args&&>(args)...));
+}
+
 // Host launchers (each returns the launch's cudaError_t).
 cudaError_t launch_router_gemm(const RouterParams& p, const CUtensorMap& tm_x, const CUtensorMap& tm_w,
                                cudaStream_t s);

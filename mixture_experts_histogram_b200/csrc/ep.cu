@@ -23,6 +23,7 @@
 
 #include "common.cuh"
 #include "moe.h"
+#include "ptx.cuh"
 
 namespace moe {
 
@@ -44,6 +45,8 @@ template <int kMaxSlots>
 __global__ void __launch_bounds__(kThreads) ep_partial_kernel(int32_t H, int32_t S, const uint16_t* __restrict__ y,
                                                               const int32_t* __restrict__ pos,
                                                               float* __restrict__ part) {
+  pdl_wait();
+  pdl_trigger();
   const int64_t t = blockIdx.x;
   int32_t rows[kMaxSlots];
 #pragma unroll
@@ -114,12 +117,9 @@ __global__ void __launch_bounds__(kThreads) ep_reduce_kernel(const ReduceParams 
 cudaError_t launch_ep_partial(int64_t T, int32_t H, int32_t S, const void* y, const int32_t* pos, float* part,
                               cudaStream_t s) {
   if (T == 0) return cudaSuccess;
-  if (S <= 9)
-    ep_partial_kernel<9><<<(unsigned)T, kThreads, 0, s>>>(H, S, static_cast<const uint16_t*>(y), pos, part);
-  else
-    ep_partial_kernel<kMaxTopK + 1><<<(unsigned)T, kThreads, 0, s>>>(H, S, static_cast<const uint16_t*>(y), pos,
-                                                                     part);
-  return counted_launch(cudaGetLastError());
+  const uint16_t* yy = static_cast<const uint16_t*>(y);
+  if (S <= 9) return launch_pdl(ep_partial_kernel<9>, dim3((unsigned)T), dim3(kThreads), 0, s, 1, H, S, yy, pos, part);
+  return launch_pdl(ep_partial_kernel<kMaxTopK + 1>, dim3((unsigned)T), dim3(kThreads), 0, s, 1, H, S, yy, pos, part);
 }
 
 }  // namespace moe

@@ -24,6 +24,8 @@ namespace moe {
 namespace {
 
 __global__ void __launch_bounds__(256) gather_bf16_kernel(const GatherParams p) {
+  pdl_wait();
+  pdl_trigger();
   const int64_t t = blockIdx.x;
   const uint4* src = reinterpret_cast<const uint4*>(p.x + t * p.H);
   const int nvec = p.H / 8;
@@ -41,6 +43,8 @@ __global__ void __launch_bounds__(256) gather_bf16_kernel(const GatherParams p) 
 // (8 bytes) to every destination row.
 template <int kMaxSlots>
 __global__ void __launch_bounds__(256) gather_fp8_kernel(const GatherParams p) {
+  pdl_wait();
+  pdl_trigger();
   const int64_t t = blockIdx.x;
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int half = lane / 16, hl = lane % 16;
@@ -96,6 +100,8 @@ __global__ void __launch_bounds__(256) gather_fp8_kernel(const GatherParams p) {
 // the sum, so up to kMaxSlots independent loads are in flight per thread.
 template <int kMaxSlots>
 __global__ void __launch_bounds__(256) combine_kernel(const CombineParams p) {
+  pdl_wait();
+  pdl_trigger();
   const int64_t t = blockIdx.x;
   const int nvec = p.H / 8;
   int32_t rows[kMaxSlots];
@@ -152,17 +158,17 @@ cudaError_t launch_scale_transpose(const float* src, float* dst, int64_t R, int3
 
 cudaError_t launch_gather(const GatherParams& p, bool fp8, cudaStream_t s) {
   if (p.T == 0) return cudaSuccess;
-  if (fp8 && p.S <= 9) gather_fp8_kernel<9><<<(unsigned)p.T, 256, 0, s>>>(p);
-  else if (fp8) gather_fp8_kernel<kMaxTopK + 1><<<(unsigned)p.T, 256, 0, s>>>(p);
-  else gather_bf16_kernel<<<(unsigned)p.T, 256, 0, s>>>(p);
-  return counted_launch(cudaGetLastError());
+  const dim3 grid((unsigned)p.T), block(256);
+  if (fp8 && p.S <= 9) return launch_pdl(gather_fp8_kernel<9>, grid, block, 0, s, 1, p);
+  if (fp8) return launch_pdl(gather_fp8_kernel<kMaxTopK + 1>, grid, block, 0, s, 1, p);
+  return launch_pdl(gather_bf16_kernel, grid, block, 0, s, 1, p);
 }
 
 cudaError_t launch_combine(const CombineParams& p, cudaStream_t s) {
   if (p.T == 0) return cudaSuccess;
-  if (p.S <= 9) combine_kernel<9><<<(unsigned)p.T, 256, 0, s>>>(p);
-  else combine_kernel<kMaxTopK + 1><<<(unsigned)p.T, 256, 0, s>>>(p);
-  return counted_launch(cudaGetLastError());
+  const dim3 grid((unsigned)p.T), block(256);
+  if (p.S <= 9) return launch_pdl(combine_kernel<9>, grid, block, 0, s, 1, p);
+  return launch_pdl(combine_kernel<kMaxTopK + 1>, grid, block, 0, s, 1, p);
 }
 
 }  // namespace moe

@@ -140,10 +140,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int unit = kPair ? (int)(blockIdx.x / 2) : (int)blockIdx.x;
   const int n_units = kPair ? (int)(gridDim.x / 2) : (int)gridDim.x;
 
-  for (int i = threadIdx.x; i <= p.G; i += kThreads) {
-    s_mt[i] = p.mt_prefix[i];
-    s_off[i] = p.offsets[i];
-  }
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::kStages; ++s) {
       mbar_init(&full[s], 1);
@@ -183,6 +179,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (kPair) cluster_sync();  // the peer's barriers are initialised before any remote arrive
   tc_fence_after_sync();
   const uint32_t tmem = *tmem_slot;
+  // Everything above overlaps the previous kernel's tail; global memory from here.
+  pdl_wait();
+  pdl_trigger();
+  for (int i = threadIdx.x; i <= p.G; i += kThreads) {
+    s_mt[i] = p.mt_prefix[i];
+    s_off[i] = p.offsets[i];
+  }
+  __syncthreads();
   const int total = s_mt[p.G] * p.n_tiles;
   const int kstages = p.K / kElemsPerStage;
   const int nkb = p.K / 128;
@@ -612,23 +616,9 @@ cudaError_t launch_one(const GemmParams& p, int grid, const AMaps& a, const CUte
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  if (!kPair) {
-    kern<<<grid, kThreads, Cfg<kPair>::kDynamic, s>>>(p, a, b0, b1, bs0, bs1);
-    return counted_launch(cudaGetLastError());
-  }
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)(grid & ~1));
-  cfg.blockDim = dim3(kThreads);
-  cfg.dynamicSmemBytes = Cfg<kPair>::kDynamic;
-  cfg.stream = s;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 2;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return counted_launch(cudaLaunchKernelEx(&cfg, kern, p, a, b0, b1, bs0, bs1));
+  if (!kPair) return launch_pdl(kern, dim3((unsigned)grid), dim3(kThreads), Cfg<kPair>::kDynamic, s, 1, p, a, b0, b1, bs0, bs1);
+  return launch_pdl(kern, dim3((unsigned)(grid & ~1)), dim3(kThreads), Cfg<kPair>::kDynamic, s, 2, p, a, b0, b1, bs0,
+                    bs1);
 }
 
 }  // namespace

@@ -136,10 +136,6 @@ __global__ void __launch_bounds__(kNvThreads, 1)
   int* s_off = reinterpret_cast<int*>(smem + L::kOff);
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  for (int i = threadIdx.x; i <= p.G; i += kNvThreads) {
-    s_mt[i] = p.mt_prefix[i];
-    s_off[i] = p.offsets[i];
-  }
   if (threadIdx.x == 0) {
     for (int s = 0; s < kConvStages; ++s) {
       mbar_init(&cfull[s], 1 + kConvWarps);  // the producer (A bytes) and every converter warp
@@ -171,6 +167,14 @@ __global__ void __launch_bounds__(kNvThreads, 1)
   __syncthreads();
   tc_fence_after_sync();
   const uint32_t tmem = *tmem_slot;
+  // Everything above overlaps the previous kernel's tail; global memory from here.
+  pdl_wait();
+  pdl_trigger();
+  for (int i = threadIdx.x; i <= p.G; i += kNvThreads) {
+    s_mt[i] = p.mt_prefix[i];
+    s_off[i] = p.offsets[i];
+  }
+  __syncthreads();
   const int total = s_mt[p.G] * p.n_tiles;
   const int kstages = p.K / 64;
   const int site0 = 0x1000 | (kGemm1 ? 0x200 : 0);  // wait-site codes recorded with a timeout
@@ -411,8 +415,7 @@ cudaError_t launch_nv(const GemmParams& p, int grid, const AMaps& a, const NvMap
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  kern<<<grid, kNvThreads, NvLayout::kDynamic, s>>>(p, a, m);
-  return counted_launch(cudaGetLastError());
+  return launch_pdl(kern, dim3((unsigned)grid), dim3(kNvThreads), NvLayout::kDynamic, s, 1, p, a, m);
 }
 
 }  // namespace

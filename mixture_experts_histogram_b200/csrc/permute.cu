@@ -44,6 +44,8 @@ __device__ __forceinline__ void histogram_block(const PermuteParams& p, int chun
 }
 
 __global__ void __launch_bounds__(256) histogram_kernel(const PermuteParams p) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ int cnt[kMaxExperts];
   histogram_block(p, blockIdx.x, cnt);
 }
@@ -108,6 +110,8 @@ __device__ __forceinline__ void scan_block(const PermuteParams& p, int* cnt_s, i
 }
 
 __global__ void __launch_bounds__(1024) scan_kernel(const PermuteParams p) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ int cnt_s[kMaxExperts + 1];
   __shared__ int off_s[kMaxExperts + 2];
   scan_block(p, cnt_s, off_s);
@@ -196,6 +200,8 @@ __device__ __forceinline__ void scatter_block(const PermuteParams& p, int chunk,
 }
 
 __global__ void __launch_bounds__(256) scatter_kernel(const PermuteParams p) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ int wcnt[8][kMaxExperts];
   scatter_block(p, blockIdx.x, wcnt);
 }
@@ -205,6 +211,8 @@ __global__ void __launch_bounds__(256) scatter_kernel(const PermuteParams p) {
 // histogram, one warp scans them over the groups, and the scatter follows. The
 // block barriers also make each step's global writes visible to the next.
 __global__ void __launch_bounds__(256) permute_one_chunk_kernel(const PermuteParams p) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ int wcnt[8][kMaxExperts];  // scatter; rows 0-1 first hold the expert counts
   int* cnt = &wcnt[0][0];
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
@@ -289,23 +297,19 @@ cudaError_t launch_tile_prefix(const int32_t* offsets, int32_t G, int32_t R, int
 }
 
 cudaError_t launch_permute_one_chunk(const PermuteParams& p, cudaStream_t s) {
-  permute_one_chunk_kernel<<<1, 256, 0, s>>>(p);
-  return counted_launch(cudaGetLastError());
+  return launch_pdl(permute_one_chunk_kernel, dim3(1), dim3(256), 0, s, 1, p);
 }
 
 cudaError_t launch_histogram(const PermuteParams& p, cudaStream_t s) {
-  histogram_kernel<<<p.chunks, 256, 0, s>>>(p);
-  return counted_launch(cudaGetLastError());
+  return launch_pdl(histogram_kernel, dim3((unsigned)p.chunks), dim3(256), 0, s, 1, p);
 }
 
 cudaError_t launch_scan(const PermuteParams& p, cudaStream_t s) {
-  scan_kernel<<<1, 1024, 0, s>>>(p);
-  return counted_launch(cudaGetLastError());
+  return launch_pdl(scan_kernel, dim3(1), dim3(1024), 0, s, 1, p);
 }
 
 cudaError_t launch_scatter(const PermuteParams& p, cudaStream_t s) {
-  scatter_kernel<<<p.chunks, 256, 0, s>>>(p);
-  return counted_launch(cudaGetLastError());
+  return launch_pdl(scatter_kernel, dim3((unsigned)p.chunks), dim3(256), 0, s, 1, p);
 }
 
 }  // namespace moe

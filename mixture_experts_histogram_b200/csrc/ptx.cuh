@@ -41,6 +41,17 @@ __device__ __forceinline__ void latch_timeout(int* status, int site, int progres
   }
 }
 
+// ------------------------------------------------ programmatic dependent launch --
+// Kernels of this library are launched with programmatic stream serialization:
+// one may start while the previous kernel in the stream is still finishing. It
+// may set up shared memory, barriers and TMEM, but must call pdl_wait() before
+// it reads or writes any global memory the previous kernel (or anything before
+// it) uses; pdl_wait returns once that kernel has completed and its writes are
+// visible. pdl_trigger() lets the next kernel start launching. Both are no-ops
+// for a kernel launched without the attribute.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // ---------------------------------------------------------------- mbarrier --
 
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {

@@ -139,6 +139,8 @@ __global__ void __launch_bounds__(kRouterThreads, 1)
   __syncthreads();
   tc_fence_after_sync();
   const uint32_t tmem = *tmem_slot;
+  pdl_wait();  // x (and the workspace) may come from the previous kernel
+  pdl_trigger();
 
   if (warp == 0 && lane == 0) {
     // ---- TMA producer ----
@@ -218,6 +220,8 @@ __global__ void __launch_bounds__(kRouterThreads, 1)
 // bias, pick the top k (largest logit first, ties to the lower index), and
 // renormalise their softmax probabilities.
 __global__ void __launch_bounds__(256) topk_kernel(const TopkParams p) {
+  pdl_wait();
+  pdl_trigger();
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int64_t t = (int64_t)blockIdx.x * 8 + warp;
   if (t >= p.T) return;
@@ -313,13 +317,11 @@ cudaError_t launch_router_gemm(const RouterParams& p, const CUtensorMap& tm_x, c
   cudaError_t e = cudaFuncSetAttribute(router_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   dim3 grid((unsigned)ceil_div(p.T, kTileM), (unsigned)p.ksplit);
-  router_gemm_kernel<<<grid, kRouterThreads, smem, s>>>(p, tm_x, tm_w);
-  return counted_launch(cudaGetLastError());
+  return launch_pdl(router_gemm_kernel, grid, dim3(kRouterThreads), smem, s, 1, p, tm_x, tm_w);
 }
 
 cudaError_t launch_topk(const TopkParams& p, cudaStream_t s) {
-  topk_kernel<<<(unsigned)ceil_div(p.T, 8), 256, 0, s>>>(p);
-  return counted_launch(cudaGetLastError());
+  return launch_pdl(topk_kernel, dim3((unsigned)ceil_div(p.T, 8)), dim3(256), 0, s, 1, p);
 }
 
 }  // namespace moe
