@@ -47,7 +47,7 @@ def parse_args():
                     default="prefill-fp8")
     ap.add_argument("--no-decode", action="store_true", help="skip the T=64 FP8 decode line")
     ap.add_argument("--no-extra", action="store_true",
-                    help="skip the Zipf-skewed T=32768 long prefill and the FP8 decode-sweep lines")
+                    help="skip the Zipf-skewed T=32768 long prefill, FP8 decode-sweep, NVFP4 and dense-FFN lines")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--residual", action="store_true",
@@ -332,7 +332,8 @@ def run_ours(args):
         # seeded weights (freed between workloads).
         for key, wshape, tokens in (("long_skew_t32768", synth.LONG_SKEW_FP8, [synth.LONG_SKEW_FP8.T]),
                                     ("decode_sweep_fp8", synth.SWEEP_FP8, list(synth.SWEEP_TOKENS)),
-                                    ("nvfp4_w4a16", synth.STEP5_NVFP4, [64, 8192])):
+                                    ("nvfp4_w4a16", synth.STEP5_NVFP4, [64, 8192]),
+                                    ("dense_ffn_fp8", synth.DENSE_FFN_FP8, [64, 8192])):
             wd = wts = None
             torch.cuda.empty_cache()
             ew = m.upload_weights(synth.make_weights(wshape), f"cuda:{local}")

@@ -27,6 +27,25 @@ constexpr int kRouterTargetCtas = 148;
 int g_gemm_variant = MOE_GEMM_AUTO;
 constexpr int64_t kPairMinRows = 128;
 
+// K pieces of the down GEMM over R rows. Its tiles (M tiles x ceil(H/256) N
+// tiles) number at most (min(G, R) + R/128) x ceil(H/256); when even that bound
+// fills less than half of the GPU (the dense FFN at decode: 16 tiles), each
+// tile's K range is split so that about one item runs per SM, every piece at
+// least 4 K stages deep, and the pieces' fp32 sums are added afterwards in
+// piece order. A function of the configuration and R only (it also sizes the
+// workspace); NVFP4 does not split.
+int down_k_split(const moe_config& c, int64_t R) {
+  if (c.wdtype == MOE_WDTYPE_NVFP4 || R <= 0) return 1;
+  const int64_t groups = c.n_experts + c.n_shared;
+  const int64_t items = ((groups < R ? groups : R) + R / kTileM) * ceil_div(c.hidden, 256);
+  if (2 * items > kRouterTargetCtas) return 1;
+  const int64_t stages = c.inter / (c.wdtype == MOE_WDTYPE_FP8_E4M3 ? 128 : 64);
+  int64_t ks = kRouterTargetCtas / items;
+  if (ks > stages / 4) ks = stages / 4;
+  if (ks > 16) ks = 16;
+  return ks < 2 ? 1 : (int)ks;
+}
+
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 std::once_flag g_encode_once;
 
@@ -309,6 +328,7 @@ int run_gate_up(const moe_config* c, const WsLayout& L, int64_t R, const void* a
     }
     if (!ok) return MOE_ERR_CUDA;
     GemmParams g{};
+  g.k_split = 1;
     g.mt_prefix = mt;
     g.offsets = offsets;
     g.G = E + S;
@@ -342,6 +362,7 @@ int run_gate_up(const moe_config* c, const WsLayout& L, int64_t R, const void* a
   }
   if (!ok) return MOE_ERR_CUDA;
   GemmParams g{};
+  g.k_split = 1;
   g.mt_prefix = pair ? mp : mt;
   g.offsets = offsets;
   g.G = E + S;
@@ -372,7 +393,7 @@ int run_gate_up(const moe_config* c, const WsLayout& L, int64_t R, const void* a
 // A [R, I] (FP8: codes with a_scale_t [I/128, rows_pad]); row_gate may be null (1).
 int run_down(const moe_config* c, const WsLayout& L, int64_t R, const void* a, const float* a_scale_t,
              const int32_t* offsets, const int32_t* mt, const int32_t* mp, bool pair, const moe_weights* w,
-             const float* row_gate, void* y, int* status, cudaStream_t s) {
+             const float* row_gate, void* y, uint8_t* ws, int* status, cudaStream_t s) {
   if (!get_encoder()) return MOE_ERR_CUDA;
   const bool fp8 = c->wdtype == MOE_WDTYPE_FP8_E4M3;
   const int H = c->hidden, I = c->inter, E = c->n_experts, S = c->n_shared;
@@ -396,6 +417,7 @@ int run_down(const moe_config* c, const WsLayout& L, int64_t R, const void* a, c
     nm.sscale1 = nm.sscale0;
     if (!ok) return MOE_ERR_CUDA;
     GemmParams g{};
+  g.k_split = 1;
     g.mt_prefix = mt;
     g.offsets = offsets;
     g.G = E + S;
@@ -429,6 +451,7 @@ int run_down(const moe_config* c, const WsLayout& L, int64_t R, const void* a, c
   }
   if (!ok) return MOE_ERR_CUDA;
   GemmParams g{};
+  g.k_split = 1;
   g.mt_prefix = pair ? mp : mt;
   g.offsets = offsets;
   g.G = E + S;
@@ -451,7 +474,11 @@ int run_down(const moe_config* c, const WsLayout& L, int64_t R, const void* a, c
   g.wait_ns = g_wait_ns;
   g.raw_out = 0;
   g.inject = g_inject;
+  g.k_split = down_k_split(*c, L.R);
+  if (g.k_split > 1) g.part = reinterpret_cast<float*>(ws + L.part);
   CUDA_TRY(launch_gemm2(g, fp8, pair, sms, ma, w2, w2h, sw2, sw2h, s));
+  if (g.k_split > 1)
+    CUDA_TRY(launch_split_reduce(g.part, g.k_split, R, H, offsets + g.G, row_gate, status, y, s));
   return MOE_OK;
 }
 
@@ -487,7 +514,7 @@ int run_experts(const moe_config* c, const WsLayout& L, int64_t T, const void* x
   if (rc != MOE_OK) return rc;
   prof.mark();
   rc = run_down(c, L, R, ws + L.h, reinterpret_cast<const float*>(ws + L.sh), offsets, mt, mp, pair2, w,
-                reinterpret_cast<const float*>(ws + L.row_gate), y, status, s);
+                reinterpret_cast<const float*>(ws + L.row_gate), y, ws, status, s);
   if (rc != MOE_OK) return rc;
   prof.mark();
   return MOE_OK;
@@ -560,6 +587,8 @@ WsLayout ws_layout(const moe_config& c, int64_t T, int target_ctas) {
   L.h = take((size_t)L.R * c.inter * es);
   L.sh = take(fp8 ? (size_t)(c.inter / 128) * L.rows_pad * 4 : 0);
   L.y = take((size_t)L.R * c.hidden * 2);
+  const int k2 = down_k_split(c, L.R);
+  L.part = take(k2 > 1 ? (size_t)k2 * L.R * c.hidden * 4 : 0);
   L.x_stage = take((size_t)T * c.hidden * 2);
   L.out_stage = take((size_t)T * c.hidden * 2);
   L.total = off;
@@ -795,7 +824,8 @@ int moe_grouped_gemm(const moe_config* cfg, int stage, int64_t R, const int32_t*
   if (stage == MOE_STAGE_DOWN) {
     float* a_t = reinterpret_cast<float*>(ws + L.sh);
     if (fp8) CUDA_TRY(launch_scale_transpose(a_scale, a_t, R, cfg->inter / 128, L.rows_pad, true, s));
-    return run_down(cfg, L, R, a, a_t, offsets, mt, mp, g_gemm_variant == MOE_GEMM_PAIR, w, row_gate, out, status, s);
+    return run_down(cfg, L, R, a, a_t, offsets, mt, mp, g_gemm_variant == MOE_GEMM_PAIR, w, row_gate, out, ws, status,
+                    s);
   }
   float* a_t = reinterpret_cast<float*>(ws + L.sxp);
   float* o_t = reinterpret_cast<float*>(ws + L.sh);

@@ -28,7 +28,7 @@ __host__ __device__ inline int64_t round_up(int64_t a, int64_t b) { return ceil_
 struct WsLayout {
   int64_t T, R, rows_pad, chunks, ksplit;
   size_t status, idx, gate, logits_part, chunk_base, counts, offsets, mt_prefix, mp_prefix;
-  size_t perm, pos, row_gate, xp, sxp, h, sh, y, x_stage, out_stage, total;
+  size_t perm, pos, row_gate, xp, sxp, h, sh, y, part, x_stage, out_stage, total;
 };
 
 WsLayout ws_layout(const moe_config& c, int64_t T, int num_sms);
@@ -112,6 +112,8 @@ struct GemmParams {
   const float* row_gate;     // GEMM2: [R]
   int* status;
   uint64_t wait_ns;          // limit of every bounded wait (normally 2 s)
+  int32_t k_split;           // K pieces per tile (>= 1; > 1 only for GEMM2, with part)
+  float* part;               // GEMM2 with k_split > 1: fp32 [k_split, R, N] piece sums, no gate
   int32_t raw_out;           // GEMM1 only: store the fp32 gate/up sums [R, 2N] instead of SwiGLU(h)
   int32_t inject;            // test hook: 1 = the producer issues no loads (the first wait runs out)
 };
@@ -207,6 +209,10 @@ cudaError_t launch_ep_partial(int64_t T, int32_t H, int32_t S, const void* y, co
 // FP8 scales between row-major [R, nb] and transposed [nb, rows_pad].
 cudaError_t launch_tile_prefix(const int32_t* offsets, int32_t G, int32_t R, int32_t* mt, int32_t* mp, int* status,
                                cudaStream_t s);
+// y [R, N] bf16 = row_gate[r] * (sum over pieces kp in order of part[kp, r, :])
+// for the rows r < min(*rows_end, R); nothing when *status is set.
+cudaError_t launch_split_reduce(const float* part, int32_t k_split, int64_t R, int32_t N, const int32_t* rows_end,
+                                const float* row_gate, const int* status, void* y, cudaStream_t s);
 cudaError_t launch_scale_transpose(const float* src, float* dst, int64_t R, int32_t nb, int64_t rows_pad,
                                    bool to_transposed, cudaStream_t s);
 

@@ -134,6 +134,35 @@ __global__ void __launch_bounds__(256) combine_kernel(const CombineParams p) {
   }
 }
 
+// Split-K down GEMM: one CTA per row; each thread sums 8 columns of the k_split
+// fp32 piece sums in piece order, applies the row's gate and rounds once.
+__global__ void __launch_bounds__(256) split_reduce_kernel(const float* __restrict__ part, int32_t k_split, int64_t R,
+                                                           int32_t N, const int32_t* __restrict__ rows_end,
+                                                           const float* __restrict__ row_gate,
+                                                           const int* __restrict__ status, uint16_t* __restrict__ y) {
+  pdl_wait();
+  pdl_trigger();
+  const int64_t r = blockIdx.x;
+  if (*status != 0) return;
+  const int64_t end = *rows_end;
+  if (r >= end) return;
+  const float g = row_gate ? row_gate[r] : 1.0f;
+  for (int c = threadIdx.x; c < N / 8; c += blockDim.x) {
+    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    for (int kp = 0; kp < k_split; ++kp) {
+      const float4* src = reinterpret_cast<const float4*>(part + ((int64_t)kp * R + r) * N) + 2 * c;
+      const float4 a = __ldcs(src), b = __ldcs(src + 1);
+      acc[0] += a.x; acc[1] += a.y; acc[2] += a.z; acc[3] += a.w;
+      acc[4] += b.x; acc[5] += b.y; acc[6] += b.z; acc[7] += b.w;
+    }
+    uint4 o;
+    __nv_bfloat162* ob = reinterpret_cast<__nv_bfloat162*>(&o);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) ob[i] = __floats2bfloat162_rn(acc[2 * i] * g, acc[2 * i + 1] * g);
+    reinterpret_cast<uint4*>(y + r * N)[c] = o;
+  }
+}
+
 // FP8 activation scales between a caller's row-major [R, nb] layout and the
 // grouped GEMMs' transposed [nb, rows_pad] one (the stage entry point).
 __global__ void __launch_bounds__(256) scale_transpose_kernel(const float* __restrict__ src, float* __restrict__ dst,
@@ -154,6 +183,13 @@ cudaError_t launch_scale_transpose(const float* src, float* dst, int64_t R, int3
   if (n == 0) return cudaSuccess;
   scale_transpose_kernel<<<(unsigned)ceil_div(n, 256), 256, 0, s>>>(src, dst, R, nb, rows_pad, to_transposed ? 1 : 0);
   return counted_launch(cudaGetLastError());
+}
+
+cudaError_t launch_split_reduce(const float* part, int32_t k_split, int64_t R, int32_t N, const int32_t* rows_end,
+                                const float* row_gate, const int* status, void* y, cudaStream_t s) {
+  if (R == 0) return cudaSuccess;
+  return launch_pdl(split_reduce_kernel, dim3((unsigned)R), dim3(256), 0, s, 1, part, k_split, R, N, rows_end, row_gate,
+                    status, static_cast<uint16_t*>(y));
 }
 
 cudaError_t launch_gather(const GatherParams& p, bool fp8, cudaStream_t s) {

@@ -187,9 +187,23 @@ __global__ void __launch_bounds__(kThreads, 1)
     s_off[i] = p.offsets[i];
   }
   __syncthreads();
-  const int total = s_mt[p.G] * p.n_tiles;
+  // Work items: (K piece, group, M tile, N tile); k_split > 1 only for the down
+  // GEMM when its tiles alone cannot fill the GPU.
+  const int base_total = s_mt[p.G] * p.n_tiles;
+  const int total = base_total * p.k_split;
   const int kstages = p.K / kElemsPerStage;
   const int nkb = p.K / 128;
+  // The item's K piece kp and K stages [ks0, ks1) (FP8: one 128-deep K block per stage).
+  auto krange = [&](int item, int& kp, int& ks0, int& ks1) {
+    kp = item / base_total;
+    ks0 = (int)((int64_t)kstages * kp / p.k_split);
+    ks1 = (int)((int64_t)kstages * (kp + 1) / p.k_split);
+  };
+  // ... and its tile.
+  auto piece = [&](int item, int& kp, int& ks0, int& ks1) -> Item {
+    krange(item, kp, ks0, ks1);
+    return decode_item(item - kp * base_total, p.n_tiles, p.G, C::kTileRows, s_mt, s_off, p.n_fastest != 0);
+  };
   const int my_off = kPair ? kTileM * (int)rank : 0;  // this CTA's rows inside a work item
   // Wait-site codes recorded with a timeout: kernel variant, CTA rank, wait.
   const int site0 = (kFP8 ? 0x100 : 0) | (kGemm1 ? 0x200 : 0) | (kPair ? 0x400 : 0) | (int)(rank << 11);
@@ -211,7 +225,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     // waits run out and the kernel returns MOE_ERR_DEVICE_TIMEOUT with nothing
     // in flight.)
     for (int item = unit; item < total && ok && p.inject != 1; item += n_units) {
-      const Item it = decode_item(item, p.n_tiles, p.G, C::kTileRows, s_mt, s_off, p.n_fastest != 0);
+      int kp, ks0, ks1;
+      const Item it = piece(item, kp, ks0, ks1);
       const bool shared = (it.g == p.E);
       const int my_row0 = it.row0 + my_off;
       const BRows<kGemm1> rows(it, p, &tm_b0, &tm_b1, &tm_bs0, &tm_bs1);
@@ -239,7 +254,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           sb1 = base + (g0 + nb1) * nkb;
         }
       }
-      for (int ks = 0; ks < kstages; ++ks) {
+      for (int ks = ks0; ks < ks1; ++ks) {
         bool w = true;
         MOE_DBG(item, ks, sc_iter);
         if (lane == 0) w = mbar_wait(&empty[stage], phase ^ 1, p.status, abort_flag, site0 | 1, item, p.wait_ns);
@@ -322,12 +337,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t acc_iter = 0;
       bool ok = true;
       for (int item = unit; item < total && ok; item += n_units) {
+        int kp, ks0, ks1;
+        krange(item, kp, ks0, ks1);
         if (!kFP8) {
           const uint32_t b = acc_iter & 1u, tph = (acc_iter >> 1) & 1u;
           if (!wait_tempty(b, tph ^ 1u, acc_iter)) { ok = false; break; }
           tc_fence_after_sync();
           const uint32_t d = tmem + b * 256;
-          for (int ks = 0; ks < kstages; ++ks) {
+          for (int ks = ks0; ks < ks1; ++ks) {
             if (!mbar_wait(&full[stage], phase, p.status, abort_flag, site0 | 4, (int)acc_iter, p.wait_ns)) {
               ok = false;
               break;
@@ -336,7 +353,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint64_t ad = sdesc_k_sw128(sA + stage * kABytes);
             const uint64_t bd = sdesc_k_sw128(sB + stage * C::kBBytes);
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk) mma(d, ad + 2 * kk, bd + 2 * kk, (ks | kk) ? 1u : 0u);
+            for (int kk = 0; kk < 4; ++kk) mma(d, ad + 2 * kk, bd + 2 * kk, (ks != ks0 || kk) ? 1u : 0u);
             commit(&empty[stage]);
             if (++stage == C::kStages) { stage = 0; phase ^= 1; }
           }
@@ -344,7 +361,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           commit(&tfull[b]);
           ++acc_iter;
         } else {
-          for (int ks = 0; ks < kstages; ++ks) {
+          for (int ks = ks0; ks < ks1; ++ks) {
             const uint32_t b = acc_iter & 1u, tph = (acc_iter >> 1) & 1u;
             MOE_DBG(item, ks, acc_iter);
             if (!wait_tempty(b, tph ^ 1u, acc_iter)) { ok = false; break; }
@@ -389,7 +406,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t acc_iter = 0, tile_iter = 0, sc_iter = 0;
     bool ok = true;
     for (int item = unit; item < total; item += n_units) {
-      const Item it = decode_item(item, p.n_tiles, p.G, C::kTileRows, s_mt, s_off, p.n_fastest != 0);
+      int kp, ks0, ks1;
+      const Item it = piece(item, kp, ks0, ks1);
       const int64_t row = (int64_t)it.row0 + my_off + rl;
       const bool row_ok = row < it.end;
       // Output columns of this thread: GEMM1 h columns n*128 + 64 hf (+64);
@@ -443,6 +461,17 @@ __global__ void __launch_bounds__(kThreads, 1)
             tmem_ld32(base + 128 * hf + 32 * ch, v);
             tmem_ld_wait();
             if (ch == 3) release_acc(b);
+            if (p.part) {
+              // Split K: this piece's fp32 sums; the gate and rounding come after the sum.
+              if (ok && row_ok && col_ok) {
+                float4* dst = reinterpret_cast<float4*>(p.part + ((int64_t)kp * p.R + row) * p.N + col0 + 32 * ch);
+#pragma unroll
+                for (int w = 0; w < 8; ++w)
+                  dst[w] = make_float4(__uint_as_float(v[4 * w]), __uint_as_float(v[4 * w + 1]),
+                                       __uint_as_float(v[4 * w + 2]), __uint_as_float(v[4 * w + 3]));
+              }
+              continue;
+            }
             uint32_t pk[16];
 #pragma unroll
             for (int i = 0; i < 16; ++i)
@@ -460,7 +489,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         float2 acc[64];
 #pragma unroll
         for (int i = 0; i < 64; ++i) acc[i] = make_float2(0.0f, 0.0f);
-        for (int kb = 0; kb < nkb; ++kb) {
+        for (int kb = ks0; kb < ks1; ++kb) {
           const uint32_t j = sc_iter % kScRing, sph = (sc_iter / kScRing) & 1u;
           MOE_DBG(item, kb, acc_iter);
           if (ok) ok = warp_wait<false>(&scfull[j], sph, p.status, abort_flag, site0 | 5, (int)sc_iter, p.wait_ns);
@@ -566,6 +595,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (hf == 0) p.out_scale[(int64_t)it.n * p.rows_pad + row] = s;
           }
           ++tile_iter;
+        } else if (p.part) {
+          // Split K: this piece's fp32 sums; the gate and rounding come after the sum.
+          if (ok && row_ok && col_ok) {
+            float4* dst = reinterpret_cast<float4*>(p.part + ((int64_t)kp * p.R + row) * p.N + col0);
+#pragma unroll
+            for (int w = 0; w < 32; ++w)
+              dst[w] = make_float4(acc[2 * w].x, acc[2 * w].y, acc[2 * w + 1].x, acc[2 * w + 1].y);
+          }
         } else {
           const float gw = row_ok ? (p.row_gate ? p.row_gate[row] : 1.0f) : 0.0f;
           if (ok && row_ok && col_ok) {

@@ -309,6 +309,14 @@ def _layer_cases():
                         seed=25), None),
         # The dense SwiGLU FFN (one expert, top-1, no shared expert, I = 13,824).
         (synth.DENSE_FFN_FP8.with_tokens(300), 12),
+        # Few down-GEMM tiles: its K range is split into pieces summed afterwards
+        # (dense FFN at T = 64 and 1: 9 pieces; the 5-group case: 2 FP8, 4 BF16).
+        (synth.DENSE_FFN_FP8.with_tokens(64), 16),
+        (synth.DENSE_FFN_FP8.with_tokens(1), None),
+        (synth.MoeShape("split-down-fp8", T=40, hidden=512, n_experts=4, top_k=1, n_shared=1, inter=1024,
+                        wdtype=synth.WDTYPE_FP8, seed=26), None),
+        (synth.MoeShape("split-down-bf16", T=40, hidden=512, n_experts=4, top_k=1, n_shared=1, inter=1024,
+                        seed=27), None),
         (dataclasses.replace(synth.DENSE_FFN_FP8, name="step5-dense-ffn-bf16", wdtype=synth.WDTYPE_BF16)
          .with_tokens(64), 8),
         (synth.DECODE_BF16, None),

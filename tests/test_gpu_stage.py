@@ -121,6 +121,39 @@ def test_down_integer_inputs_bit_exact(m, fp8, variant):
     assert bad.size == 0, f"{len(bad)} outputs differ, first {bad[:4].tolist()}"
 
 
+@pytest.mark.parametrize("fp8", [True, False], ids=["fp8", "bf16"])
+def test_down_split_k_integer_inputs_bit_exact(m, fp8, variant):
+    """One group of 50 rows under a 64-row call, K = 2048, H = 512: two output
+    tiles for the whole GPU, so the down GEMM splits K (4 pieces FP8, 8 BF16)
+    and sums the pieces afterwards; integer sums stay exact in any order, and
+    the 14 rows past the group's end are left untouched."""
+    import torch
+    h, i2, r, valid = 512, 2048, 64, 50
+    wd = synth.WDTYPE_FP8 if fp8 else synth.WDTYPE_BF16
+    cfg = m.make_config(h, 1, 1, 0, i2, wd)
+    w1, w3, w2 = _ints(11, (1, i2, h)), _ints(12, (1, i2, h)), _ints(13, (1, h, i2))
+    host = {"router_w": synth.normal_bf16(0, 1, (1, h), 0.05), "router_bias": None,
+            "w1": _codes(w1, fp8), "w3": _codes(w3, fp8), "w2": _codes(w2, fp8),
+            "s1": np.ones((1, i2 // 128, h // 128), np.float32) if fp8 else None,
+            "s3": np.ones((1, i2 // 128, h // 128), np.float32) if fp8 else None,
+            "s2": np.ones((1, h // 128, i2 // 128), np.float32) if fp8 else None}
+    dev = m.upload_weights(host)
+    ws = torch.empty(m.moe_workspace_bytes(cfg, r), dtype=torch.uint8, device="cuda")
+    a = _ints(14, (r, i2))
+    gate = np.random.default_rng(15).choice(np.array([0.25, 0.5, 1.0, 2.0], np.float32), size=r)
+    y = torch.full((r, h), 7.0, dtype=torch.bfloat16, device="cuda")
+    a_scale = m.to_device(np.ones((r, i2 // 128), np.float32)) if fp8 else None
+    m.moe_grouped_gemm(cfg, m.MOE_STAGE_DOWN, r, m.to_device(np.array([0, valid], np.int32)),
+                       m.to_device(_codes(a, fp8)), a_scale, m.make_weights(dev), y, ws, row_gate=m.to_device(gate))
+    assert m.moe_read_status(ws) == 0
+    got = y.view(torch.int16).cpu().numpy().view(np.uint16)
+    ref = (a[:valid] @ w2[0].T).astype(np.float64) * gate[:valid, None].astype(np.float64)
+    assert np.abs(ref).max() < 2 ** 24
+    bad = np.argwhere(got[:valid] != synth.f32_to_bf16(ref.astype(np.float32)))
+    assert bad.size == 0, f"{len(bad)} outputs differ, first {bad[:4].tolist()}"
+    assert (got[valid:] == synth.f32_to_bf16(np.float32(7.0))).all()
+
+
 def test_grouped_gemm_rejects_bad_offsets(m):
     import torch
     cfg, dev, _, offsets, R, _, ws = _setup(m, True)
