@@ -336,11 +336,15 @@ MOE_API const char* moe_profile_kernel_name(int i);
 
 /* Expert-GEMM variant (process-wide; default MOE_GEMM_AUTO). SINGLE runs one
  * CTA per 128-row tile; PAIR runs 2-SM CTA pairs on 256-row tiles (each weight
- * tile crosses L2 -> SM once per 256 rows). AUTO runs the gate/up GEMM on pairs
- * when top_k * T >= 128 * n_experts (routed groups of 128+ rows on average) and
- * everything else on single CTAs. All variants compute the same layer and are
- * held to the same tolerance by the tests. */
-enum { MOE_GEMM_AUTO = 0, MOE_GEMM_SINGLE = 1, MOE_GEMM_PAIR = 2 };
+ * tile crosses L2 -> SM once per 256 rows); SWAP (FP8 storage only; others run
+ * SINGLE) makes the weight rows the MMA's M side and runs each group in chunks
+ * of 32 rows, for decode-sized groups. AUTO runs both FP8 GEMMs swapped when
+ * n_experts <= top_k * T <= 16 * n_experts, else the gate/up GEMM on pairs when
+ * top_k * T >= 128 * n_experts (routed groups of 128+ rows on average) and
+ * everything else on single CTAs. The stage entry point applies the same rules
+ * with its R rows and n_experts + n_shared groups. All variants compute the
+ * same layer and are held to the same tolerance by the tests. */
+enum { MOE_GEMM_AUTO = 0, MOE_GEMM_SINGLE = 1, MOE_GEMM_PAIR = 2, MOE_GEMM_SWAP = 3 };
 MOE_API int moe_set_gemm_variant(int variant);
 
 /* Kernels this library has launched in this process so far (every entry

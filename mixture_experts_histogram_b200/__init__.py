@@ -31,7 +31,7 @@ MOE_ERR_CUDA = 4
 MOE_ERR_BAD_INDEX = 5
 MOE_ERR_DEVICE_TIMEOUT = 6
 MOE_ERR_MISALIGNED = 7
-MOE_GEMM_AUTO, MOE_GEMM_SINGLE, MOE_GEMM_PAIR = 0, 1, 2
+MOE_GEMM_AUTO, MOE_GEMM_SINGLE, MOE_GEMM_PAIR, MOE_GEMM_SWAP = 0, 1, 2, 3
 MOE_STAGE_GATE_UP, MOE_STAGE_GATE_UP_RAW, MOE_STAGE_DOWN = 1, 2, 3
 MOE_INJECT_NONE, MOE_INJECT_GEMM_NO_LOADS = 0, 1
 

@@ -26,6 +26,8 @@ constexpr int kRouterTargetCtas = 148;
 // which measured faster at every size (0.91 vs 0.98 ms at T = 8192).
 int g_gemm_variant = MOE_GEMM_AUTO;
 constexpr int64_t kPairMinRows = 128;
+constexpr int64_t kSwapMinRows = 1;
+constexpr int64_t kSwapMaxRows = 16;
 
 // K pieces of the down GEMM over R rows. Its tiles (M tiles x ceil(H/256) N
 // tiles) number at most (min(G, R) + R/128) x ceil(H/256); when even that bound
@@ -283,11 +285,26 @@ int run_permute(const PermuteParams& pp, cudaStream_t s, Prof& prof) {
 uint64_t g_wait_ns = kWaitLimitNs;
 int g_inject = 0;
 
-// GEMM1 runs on 2-SM pairs under AUTO when the routed groups average at least
-// kPairMinRows rows.
-bool gate_up_on_pairs(int64_t routed_rows, int n_experts) {
-  return g_gemm_variant == MOE_GEMM_PAIR ||
-         (g_gemm_variant == MOE_GEMM_AUTO && routed_rows >= kPairMinRows * (int64_t)n_experts);
+// Kernel of one expert GEMM: single CTAs, 2-SM pairs, or (FP8) the swapped-
+// operand kernel for decode-sized groups. Under AUTO, FP8 layers whose routed
+// groups average kSwapMinRows to kSwapMaxRows rows run both GEMMs swapped
+// (T = 64: GEMM1 0.580 -> 0.563 ms, GEMM2 0.302 -> 0.282; T = 512 about equal;
+// at T <= 8 the single-CTA kernel was 5-8% faster); otherwise GEMM1 runs on
+// pairs when the groups average at least kPairMinRows rows and GEMM2 on
+// single CTAs.
+enum GemmKind { kSingle = 0, kPair = 1, kSwap = 2 };
+
+GemmKind gemm_kind(bool gate_up, int64_t routed_rows, int n_experts, int wdtype) {
+  const bool fp8 = wdtype == MOE_WDTYPE_FP8_E4M3;
+  switch (g_gemm_variant) {
+    case MOE_GEMM_SINGLE: return kSingle;
+    case MOE_GEMM_PAIR: return kPair;
+    case MOE_GEMM_SWAP: return fp8 ? kSwap : kSingle;
+    default: break;
+  }
+  if (fp8 && routed_rows >= kSwapMinRows * (int64_t)n_experts && routed_rows <= kSwapMaxRows * (int64_t)n_experts)
+    return kSwap;
+  return (gate_up && routed_rows >= kPairMinRows * (int64_t)n_experts) ? kPair : kSingle;
 }
 
 bool amaps(AMaps* a, const void* base, bool fp8, uint64_t inner, uint64_t rows) {
@@ -301,8 +318,9 @@ bool amaps(AMaps* a, const void* base, bool fp8, uint64_t inner, uint64_t rows) 
 // rows_pad]; out = h codes [R, I] with out_scale_t [I/128, rows_pad]. BF16: out
 // = h [R, I] bf16. raw: out = fp32 [R, 2I] gate and up sums (no SwiGLU).
 int run_gate_up(const moe_config* c, const WsLayout& L, int64_t R, const void* a, const float* a_scale_t,
-                const int32_t* offsets, const int32_t* mt, const int32_t* mp, bool pair, const moe_weights* w,
+                const int32_t* offsets, const int32_t* mt, const int32_t* mp, GemmKind kind, const moe_weights* w,
                 void* out, float* out_scale_t, bool raw, int* status, cudaStream_t s) {
+  const bool pair = kind == kPair;
   if (!get_encoder()) return MOE_ERR_CUDA;
   const bool fp8 = c->wdtype == MOE_WDTYPE_FP8_E4M3;
   const int H = c->hidden, I = c->inter, E = c->n_experts, S = c->n_shared;
@@ -385,15 +403,17 @@ int run_gate_up(const moe_config* c, const WsLayout& L, int64_t R, const void* a
   g.wait_ns = g_wait_ns;
   g.raw_out = raw ? 1 : 0;
   g.inject = g_inject;
-  CUDA_TRY(launch_gemm1(g, fp8, pair, sms, ma, w1, w3, sw1, sw3, s));
+  if (kind == kSwap && fp8) CUDA_TRY(launch_gemm_swap(g, true, sms, ma, w1, w3, sw1, sw3, s));
+  else CUDA_TRY(launch_gemm1(g, fp8, pair, sms, ma, w1, w3, sw1, sw3, s));
   return MOE_OK;
 }
 
 // The grouped down GEMM (GEMM2): y [R, H] bf16 = row_gate[r] * (A W2_g^T) for
 // A [R, I] (FP8: codes with a_scale_t [I/128, rows_pad]); row_gate may be null (1).
 int run_down(const moe_config* c, const WsLayout& L, int64_t R, const void* a, const float* a_scale_t,
-             const int32_t* offsets, const int32_t* mt, const int32_t* mp, bool pair, const moe_weights* w,
+             const int32_t* offsets, const int32_t* mt, const int32_t* mp, GemmKind kind, const moe_weights* w,
              const float* row_gate, void* y, uint8_t* ws, int* status, cudaStream_t s) {
+  const bool pair = kind == kPair;
   if (!get_encoder()) return MOE_ERR_CUDA;
   const bool fp8 = c->wdtype == MOE_WDTYPE_FP8_E4M3;
   const int H = c->hidden, I = c->inter, E = c->n_experts, S = c->n_shared;
@@ -476,7 +496,8 @@ int run_down(const moe_config* c, const WsLayout& L, int64_t R, const void* a, c
   g.inject = g_inject;
   g.k_split = down_k_split(*c, L.R);
   if (g.k_split > 1) g.part = reinterpret_cast<float*>(ws + L.part);
-  CUDA_TRY(launch_gemm2(g, fp8, pair, sms, ma, w2, w2h, sw2, sw2h, s));
+  if (kind == kSwap && fp8) CUDA_TRY(launch_gemm_swap(g, false, sms, ma, w2, w2h, sw2, sw2h, s));
+  else CUDA_TRY(launch_gemm2(g, fp8, pair, sms, ma, w2, w2h, sw2, sw2h, s));
   if (g.k_split > 1)
     CUDA_TRY(launch_split_reduce(g.part, g.k_split, R, H, offsets + g.G, row_gate, status, y, s));
   return MOE_OK;
@@ -507,13 +528,13 @@ int run_experts(const moe_config* c, const WsLayout& L, int64_t T, const void* x
   const int32_t* mt = reinterpret_cast<const int32_t*>(ws + L.mt_prefix);
   const int32_t* mp = reinterpret_cast<const int32_t*>(ws + L.mp_prefix);
   int* status = reinterpret_cast<int*>(ws + L.status);
-  const bool pair2 = g_gemm_variant == MOE_GEMM_PAIR;
-  const bool pair1 = gate_up_on_pairs(routed_rows, c->n_experts);
-  int rc = run_gate_up(c, L, R, ws + L.xp, reinterpret_cast<const float*>(ws + L.sxp), offsets, mt, mp, pair1, w,
+  const GemmKind k1 = gemm_kind(true, routed_rows, c->n_experts, c->wdtype);
+  const GemmKind k2 = gemm_kind(false, routed_rows, c->n_experts, c->wdtype);
+  int rc = run_gate_up(c, L, R, ws + L.xp, reinterpret_cast<const float*>(ws + L.sxp), offsets, mt, mp, k1, w,
                        ws + L.h, reinterpret_cast<float*>(ws + L.sh), false, status, s);
   if (rc != MOE_OK) return rc;
   prof.mark();
-  rc = run_down(c, L, R, ws + L.h, reinterpret_cast<const float*>(ws + L.sh), offsets, mt, mp, pair2, w,
+  rc = run_down(c, L, R, ws + L.h, reinterpret_cast<const float*>(ws + L.sh), offsets, mt, mp, k2, w,
                 reinterpret_cast<const float*>(ws + L.row_gate), y, ws, status, s);
   if (rc != MOE_OK) return rc;
   prof.mark();
@@ -824,14 +845,15 @@ int moe_grouped_gemm(const moe_config* cfg, int stage, int64_t R, const int32_t*
   if (stage == MOE_STAGE_DOWN) {
     float* a_t = reinterpret_cast<float*>(ws + L.sh);
     if (fp8) CUDA_TRY(launch_scale_transpose(a_scale, a_t, R, cfg->inter / 128, L.rows_pad, true, s));
-    return run_down(cfg, L, R, a, a_t, offsets, mt, mp, g_gemm_variant == MOE_GEMM_PAIR, w, row_gate, out, ws, status,
-                    s);
+    return run_down(cfg, L, R, a, a_t, offsets, mt, mp, gemm_kind(false, R, G, cfg->wdtype), w, row_gate, out, ws,
+                    status, s);
   }
   float* a_t = reinterpret_cast<float*>(ws + L.sxp);
   float* o_t = reinterpret_cast<float*>(ws + L.sh);
   if (fp8) CUDA_TRY(launch_scale_transpose(a_scale, a_t, R, cfg->hidden / 128, L.rows_pad, true, s));
   const bool raw = stage == MOE_STAGE_GATE_UP_RAW;
-  rc = run_gate_up(cfg, L, R, a, a_t, offsets, mt, mp, gate_up_on_pairs(R, G), w, out, o_t, raw, status, s);
+  rc = run_gate_up(cfg, L, R, a, a_t, offsets, mt, mp, gemm_kind(true, R, G, cfg->wdtype), w, out, o_t, raw, status,
+                   s);
   if (rc != MOE_OK) return rc;
   if (fp8 && !raw) CUDA_TRY(launch_scale_transpose(o_t, out_scale, R, cfg->inter / 128, L.rows_pad, false, s));
   return MOE_OK;
@@ -899,7 +921,8 @@ int moe_profile_read(float* ms, int n, int* n_out) {
 const char* moe_profile_kernel_name(int i) { return (i >= 0 && i < kProfKernels) ? kProfNames[i] : ""; }
 
 int moe_set_gemm_variant(int variant) {
-  if (variant != MOE_GEMM_AUTO && variant != MOE_GEMM_SINGLE && variant != MOE_GEMM_PAIR) return MOE_ERR_INVALID_ARG;
+  if (variant != MOE_GEMM_AUTO && variant != MOE_GEMM_SINGLE && variant != MOE_GEMM_PAIR && variant != MOE_GEMM_SWAP)
+    return MOE_ERR_INVALID_ARG;
   g_gemm_variant = variant;
   return MOE_OK;
 }

@@ -127,6 +127,10 @@ def test_grouped_gemm_and_hooks_argument_errors_need_no_device(lib):
              1 << 20, None) == m.MOE_OK                                                    # R = 0: no-op
     assert lib.moe_debug_inject(7, 0) == m.MOE_ERR_INVALID_ARG
     assert lib.moe_debug_inject(m.MOE_INJECT_NONE, 0) == m.MOE_OK
+    for v in (m.MOE_GEMM_SINGLE, m.MOE_GEMM_PAIR, m.MOE_GEMM_SWAP, m.MOE_GEMM_AUTO):
+        assert lib.moe_set_gemm_variant(v) == m.MOE_OK
+    assert lib.moe_set_gemm_variant(4) == m.MOE_ERR_INVALID_ARG
+    assert lib.moe_set_gemm_variant(-1) == m.MOE_ERR_INVALID_ARG
 
 
 def test_expert_parallel_argument_errors_need_no_device(lib):

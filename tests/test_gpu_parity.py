@@ -257,10 +257,10 @@ def _expert_cases():
     ]
 
 
-@pytest.fixture(params=["single", "pair"])
+@pytest.fixture(params=["single", "pair", "swap"])
 def variant(request, m):
     """Run the test under each expert-GEMM variant (same result expected)."""
-    m.moe_set_gemm_variant(m.MOE_GEMM_SINGLE if request.param == "single" else m.MOE_GEMM_PAIR)
+    m.moe_set_gemm_variant({"single": m.MOE_GEMM_SINGLE, "pair": m.MOE_GEMM_PAIR, "swap": m.MOE_GEMM_SWAP}[request.param])
     yield request.param
     m.moe_set_gemm_variant(m.MOE_GEMM_AUTO)
 

@@ -7,7 +7,8 @@ the integer result bit for bit. The expected values are the plain definition
 (an int64 matrix product per group); the gate/up GEMM is read before its
 SwiGLU (MOE_STAGE_GATE_UP_RAW), the down GEMM through its bf16 output with
 power-of-two row gates (one exact scaling, then one round-to-nearest-even).
-Both GEMM variants (single CTAs, 2-SM pairs) run the same rows.
+Every GEMM variant (single CTAs, 2-SM pairs, and for FP8 the swapped-operand
+kernel that runs groups in 32-row chunks) runs the same rows.
 
 Bounded waits: moe_debug_inject(MOE_INJECT_GEMM_NO_LOADS) makes the expert
 GEMMs' producer issue no loads, so their consumers' waits run out; the call
@@ -34,9 +35,9 @@ def m():
     return mm
 
 
-@pytest.fixture(params=["single", "pair"])
+@pytest.fixture(params=["single", "pair", "swap"])
 def variant(request, m):
-    m.moe_set_gemm_variant(m.MOE_GEMM_SINGLE if request.param == "single" else m.MOE_GEMM_PAIR)
+    m.moe_set_gemm_variant({"single": m.MOE_GEMM_SINGLE, "pair": m.MOE_GEMM_PAIR, "swap": m.MOE_GEMM_SWAP}[request.param])
     yield request.param
     m.moe_set_gemm_variant(m.MOE_GEMM_AUTO)
 
