@@ -336,10 +336,12 @@ MOE_API const char* moe_profile_kernel_name(int i);
 
 /* Expert-GEMM variant (process-wide; default MOE_GEMM_AUTO). SINGLE runs one
  * CTA per 128-row tile; PAIR runs 2-SM CTA pairs on 256-row tiles (each weight
- * tile crosses L2 -> SM once per 256 rows); SWAP (FP8 storage only; others run
- * SINGLE) makes the weight rows the MMA's M side and runs each group in chunks
- * of 32 rows, for decode-sized groups. AUTO runs both FP8 GEMMs swapped when
- * n_experts <= top_k * T <= 16 * n_experts, else the gate/up GEMM on pairs when
+ * tile crosses L2 -> SM once per 256 rows; NVFP4 runs SINGLE); SWAP (FP8 and
+ * NVFP4 storage; BF16 runs SINGLE) makes the weight rows the MMA's M side and
+ * runs each group in chunks of 32 rows, for decode-sized groups (NVFP4: the
+ * weights expanded into tensor memory). AUTO runs both FP8 GEMMs swapped when
+ * n_experts <= top_k * T <= 16 * n_experts and both NVFP4 GEMMs swapped when
+ * top_k * T <= 16 * n_experts, else the gate/up GEMM on pairs when
  * top_k * T >= 128 * n_experts (routed groups of 128+ rows on average) and
  * everything else on single CTAs. The stage entry point applies the same rules
  * with its R rows and n_experts + n_shared groups. All variants compute the

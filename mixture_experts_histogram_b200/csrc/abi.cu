@@ -296,12 +296,14 @@ enum GemmKind { kSingle = 0, kPair = 1, kSwap = 2 };
 
 GemmKind gemm_kind(bool gate_up, int64_t routed_rows, int n_experts, int wdtype) {
   const bool fp8 = wdtype == MOE_WDTYPE_FP8_E4M3;
+  const bool nvfp4 = wdtype == MOE_WDTYPE_NVFP4;
   switch (g_gemm_variant) {
     case MOE_GEMM_SINGLE: return kSingle;
-    case MOE_GEMM_PAIR: return kPair;
-    case MOE_GEMM_SWAP: return fp8 ? kSwap : kSingle;
+    case MOE_GEMM_PAIR: return nvfp4 ? kSingle : kPair;
+    case MOE_GEMM_SWAP: return (fp8 || nvfp4) ? kSwap : kSingle;
     default: break;
   }
+  if (nvfp4) return routed_rows <= kSwapMaxRows * (int64_t)n_experts ? kSwap : kSingle;
   if (fp8 && routed_rows >= kSwapMinRows * (int64_t)n_experts && routed_rows <= kSwapMaxRows * (int64_t)n_experts)
     return kSwap;
   return (gate_up && routed_rows >= kPairMinRows * (int64_t)n_experts) ? kPair : kSingle;
@@ -366,7 +368,8 @@ int run_gate_up(const moe_config* c, const WsLayout& L, int64_t R, const void* a
     g.wait_ns = g_wait_ns;
     g.raw_out = raw ? 1 : 0;
     g.inject = g_inject;
-    CUDA_TRY(launch_nvfp4_gemm(g, true, sms, ma, nm, s));
+    if (kind == kSwap) CUDA_TRY(launch_nvfp4_swap(g, true, sms, ma, nm, s));
+    else CUDA_TRY(launch_nvfp4_gemm(g, true, sms, ma, nm, s));
     return MOE_OK;
   }
   CUtensorMap w1, w3, sw1, sw3;
@@ -457,7 +460,8 @@ int run_down(const moe_config* c, const WsLayout& L, int64_t R, const void* a, c
     g.status = status;
     g.wait_ns = g_wait_ns;
     g.inject = g_inject;
-    CUDA_TRY(launch_nvfp4_gemm(g, false, sms, ma, nm, s));
+    if (kind == kSwap) CUDA_TRY(launch_nvfp4_swap(g, false, sms, ma, nm, s));
+    else CUDA_TRY(launch_nvfp4_gemm(g, false, sms, ma, nm, s));
     return MOE_OK;
   }
   CUtensorMap w2, w2h, sw2, sw2h;

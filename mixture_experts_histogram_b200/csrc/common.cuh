@@ -197,6 +197,11 @@ cudaError_t launch_gemm1(const GemmParams& p, bool fp8, bool pair, int grid, con
                          const CUtensorMap& tm_w1, const CUtensorMap& tm_w3, const CUtensorMap& tm_sw1,
                          const CUtensorMap& tm_sw3, cudaStream_t s);
 // tm_w2 / tm_sw2 use 256-row boxes, tm_w2h / tm_sw2h the same tensors with 128-row boxes.
+// The NVFP4 GEMMs for decode-sized groups (nvfp4_gemm_swap.cu): weights expanded
+// into TMEM as the MMA's A operand, a group's rows as N in 32-row chunks; maps
+// and parameters as for launch_nvfp4_gemm (p.mt_prefix not used).
+cudaError_t launch_nvfp4_swap(const GemmParams& p, bool gemm1, int grid, const AMaps& tm_a, const NvMaps& tm,
+                              cudaStream_t s);
 // The swapped-operand FP8 GEMMs for decode-sized groups (grouped_gemm_swap.cu):
 // GEMM1 (gemm1: b0/b1 = W1/W3 with 128-row boxes) or GEMM2 (b0 = W2 with
 // 256-row boxes); p.mt_prefix is not used (the kernel derives its 32-row chunks

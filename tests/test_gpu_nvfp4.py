@@ -7,7 +7,9 @@ scales make every weight a small dyadic number, and bf16 activations in
 definition bit for bit; this pins the codes' nibble order, the scale indexing,
 the shared-memory layout the converter warps write and the global scales.
 Then the whole layer against the oracle on seeded NVFP4 weights, within the
-BF16 tolerance 1e-2 (relative Frobenius, pooled and per token).
+BF16 tolerance 1e-2 (relative Frobenius, pooled and per token). Every case runs
+both NVFP4 kernels (128-row tiles, and weight rows as the MMA's M side with the
+weights expanded into tensor memory).
 """
 import numpy as np
 import pytest
@@ -29,6 +31,15 @@ def m():
     build.build()
     mm.load()
     return mm
+
+
+@pytest.fixture(params=["single", "swap"])
+def variant(request, m):
+    """The NVFP4 GEMM kernels: tiles of 128 rows, or weight rows as the MMA's M side
+    expanded into tensor memory (same results expected)."""
+    m.moe_set_gemm_variant(m.MOE_GEMM_SINGLE if request.param == "single" else m.MOE_GEMM_SWAP)
+    yield request.param
+    m.moe_set_gemm_variant(m.MOE_GEMM_AUTO)
 
 
 H, I, E = 512, 256, 5
@@ -71,7 +82,7 @@ def _setup(m):
     return cfg, dev, (w1, w3, w2), offsets, R, group, ws
 
 
-def test_nvfp4_gate_up_exact(m):
+def test_nvfp4_gate_up_exact(m, variant):
     import torch
     cfg, dev, (w1, w3, _), offsets, R, group, ws = _setup(m)
     a = np.random.default_rng(4).integers(-4, 5, size=(R, H)).astype(np.float64)
@@ -90,7 +101,7 @@ def test_nvfp4_gate_up_exact(m):
     assert bad.size == 0, f"{len(bad)} sums differ, first {bad[:4].tolist()}"
 
 
-def test_nvfp4_down_exact(m):
+def test_nvfp4_down_exact(m, variant):
     import torch
     cfg, dev, (_, _, w2), offsets, R, group, ws = _setup(m)
     a = np.random.default_rng(5).integers(-4, 5, size=(R, I)).astype(np.float64)
@@ -125,7 +136,7 @@ LAYER_CASES = [
 
 
 @pytest.mark.parametrize("shape,n_sample", LAYER_CASES, ids=lambda v: getattr(v, "name", str(v)))
-def test_nvfp4_layer_parity(m, shape, n_sample):
+def test_nvfp4_layer_parity(m, shape, n_sample, variant):
     import torch
     x, w = synth.make_x(shape), synth.make_weights(shape)
     idx_r, gate_r, logits_r = oracle.route(x, w["router_w"], w["router_bias"], shape.top_k, want_logits=True)
