@@ -24,8 +24,10 @@
 //   warps 2-5   epilogue: warp w reads TMEM lane quarter w % 4 of both
 //               accumulators (one weight row per thread; GEMM1: its gate and up
 //               sums side by side) for the chunk's 32 rows.
-//   warps 6-9   converters: warp w expands weight rows 32 (w % 4) + lane of both
-//               128-row halves of the tile into that lane's TMEM columns.
+//   warps 6-13  converters: warp w expands weight row 32 (w % 4) + lane of the
+//               tile's 128-row half (w - 6) / 4 into that lane's TMEM columns
+//               (two converter warps per SM sub-partition: the expansion is
+//               latency-bound with one).
 // TMEM columns: [0, 128) two accumulator buffers of 2 x 32 columns (tile half 0
 // rows, then half 1); [128, 128 + 64 kAStages) the A stages, 32 columns per
 // half (K elements 2c, 2c + 1 in column c).
@@ -40,7 +42,7 @@ namespace moe {
 namespace {
 
 constexpr int kNsEpiWarps = 4;
-constexpr int kNsConvWarps = 4;
+constexpr int kNsConvWarps = 8;
 constexpr int kNsThreads = 32 * (2 + kNsEpiWarps + kNsConvWarps);
 constexpr int kNsTok = 32;                       // rows per chunk (MMA N)
 constexpr int kNsRaw = 8;                        // code stages in flight
@@ -72,8 +74,11 @@ struct NsLayout {
   static_assert(kDynamic <= 227 * 1024, "shared memory budget");
 };
 
+// 14 warps put four on two of the SM's sub-partitions, whose register files
+// then allow 128 registers a thread: the bound is declared for 512 threads.
+static_assert(kNsThreads <= 512, "register budget");
 template <bool kGemm1>
-__global__ void __launch_bounds__(kNsThreads, 1)
+__global__ void __launch_bounds__(512, 1)
     nvfp4_swap_kernel(const GemmParams p, const __grid_constant__ AMaps tm_a, const __grid_constant__ NvMaps tm) {
   using L = NsLayout;
   constexpr uint32_t kIdesc = idesc_mma(1u, 128, kNsTok);  // bf16 x bf16, M = 128, N = 32
@@ -320,9 +325,10 @@ __global__ void __launch_bounds__(kNsThreads, 1)
     }
   } else {
     // --------------------------------------------------------- converters --
-    // Thread: weight row wrow of half 0 (raw row wrow) and of half 1 (raw row
-    // 128 + wrow), 64 K elements each per stage, into TMEM lane wrow.
+    // Thread: weight row wrow of half h (raw row 128 h + wrow), 64 K elements
+    // per stage, into TMEM lane wrow.
     const int q = warp % 4;
+    const int h = (warp - 2 - kNsEpiWarps) / 4;
     const int wrow = 32 * q + lane;
     const uint32_t lane_base = (uint32_t)(q * 32) << 16;
     uint32_t it_raw = 0, it_a = 0;
@@ -339,8 +345,7 @@ __global__ void __launch_bounds__(kNsThreads, 1)
         tc_fence_after_sync();
         const uint8_t* codes = sCodes + rs * kNsCodeBytes;
         const uint8_t* scl = sScales + ((it_raw / 4) % kNsScaleSlots) * kNsScaleBytes + (ks & 3) * 4;
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
+        {
           const int rr = 128 * h + wrow;
           const uint4 w0 = *reinterpret_cast<const uint4*>(codes + rr * 32);
           const uint4 w1 = *reinterpret_cast<const uint4*>(codes + rr * 32 + 16);
