@@ -512,9 +512,10 @@ def traffic_for(kernel: str, workload_name: str):
         return None
 
 
-# Sources that build the FP8 grouped GEMMs and their launch (tensor maps,
+# Sources that build the grouped expert GEMMs and their launch (tensor maps,
 # variant choice): the files a traffic figure for those kernels depends on.
-GEMM_SOURCES = ("grouped_gemm.cu", "grouped_gemm_swap.cu", "gemm_common.cuh", "ptx.cuh", "common.cuh", "abi.cu")
+GEMM_SOURCES = ("grouped_gemm.cu", "grouped_gemm_swap.cu", "nvfp4_gemm.cu", "nvfp4_gemm_swap.cu", "gemm_common.cuh",
+                "ptx.cuh", "common.cuh", "abi.cu")
 
 
 def kernel_source_sha() -> str:
