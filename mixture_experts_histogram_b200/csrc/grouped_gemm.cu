@@ -425,7 +425,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t g[32], u[32];
             tmem_ld32(base + 64 * hf + 32 * ch, g);
             tmem_ld32(base + 128 + 64 * hf + 32 * ch, u);
-            tmem_ld_wait();
+            tmem_ld_wait(g);
+            tmem_ld_wait(u);
             if (ch == 1) release_acc(b);
             if (p.raw_out) {
               // The fp32 gate and up sums themselves (stage entry point, tests).
@@ -459,7 +460,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int ch = 0; ch < 4; ++ch) {
             uint32_t v[32];
             tmem_ld32(base + 128 * hf + 32 * ch, v);
-            tmem_ld_wait();
+            tmem_ld_wait(v);
             if (ch == 3) release_acc(b);
             if (p.part) {
               // Split K: this piece's fp32 sums; the gate and rounding come after the sum.

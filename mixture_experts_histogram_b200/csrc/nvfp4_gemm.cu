@@ -277,7 +277,8 @@ __global__ void __launch_bounds__(kNvThreads, 1)
           uint32_t g[32], u[32];
           tmem_ld32(base + 64 * hf + 32 * ch, g);
           tmem_ld32(base + 128 + 64 * hf + 32 * ch, u);
-          tmem_ld_wait();
+          tmem_ld_wait(g);
+          tmem_ld_wait(u);
           if (ch == 1) release();
           if (p.raw_out) {
             if (ok && row_ok) {
@@ -311,7 +312,7 @@ __global__ void __launch_bounds__(kNvThreads, 1)
         for (int ch = 0; ch < 4; ++ch) {
           uint32_t v[32];
           tmem_ld32(base + 128 * hf + 32 * ch, v);
-          tmem_ld_wait();
+          tmem_ld_wait(v);
           if (ch == 3) release();
           uint32_t pk[16];
 #pragma unroll

@@ -390,6 +390,8 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
       : "r"(taddr));
 }
 
+// The wait for every earlier tcgen05.ld of the thread. Prefer the overloads
+// below, which name the loaded registers so no use of them is scheduled earlier.
 __device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
 // The same wait, naming the registers of an earlier tcgen05.ld as read and

@@ -55,7 +55,7 @@ __device__ __forceinline__ void fused_topk(const RouterParams& p, uint32_t taddr
   for (int c0 = 0; c0 < ncols; c0 += 32) {
     uint32_t v[32];
     tmem_ld32(taddr + (uint32_t)c0, v);
-    tmem_ld_wait();
+    tmem_ld_wait(v);
 #pragma unroll
     for (int i = 0; i < 32; ++i) {
       const int e = c0 + i;
@@ -197,7 +197,7 @@ __global__ void __launch_bounds__(kRouterThreads, 1)
       for (int c0 = 0; c0 < ncols; c0 += 32) {
         uint32_t v[32];
         tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)c0, v);
-        tmem_ld_wait();
+        tmem_ld_wait(v);
 #pragma unroll
         for (int i = 0; i < 32; ++i) tr[lane * 33 + i] = __uint_as_float(v[i]);
         __syncwarp();
