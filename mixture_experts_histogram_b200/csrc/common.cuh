@@ -196,7 +196,9 @@ cudaError_t launch_nvfp4_gemm(const GemmParams& p, bool gemm1, int grid, const A
 cudaError_t launch_gemm1(const GemmParams& p, bool fp8, bool pair, int grid, const AMaps& tm_a,
                          const CUtensorMap& tm_w1, const CUtensorMap& tm_w3, const CUtensorMap& tm_sw1,
                          const CUtensorMap& tm_sw3, cudaStream_t s);
-// tm_w2 / tm_sw2 use 256-row boxes, tm_w2h / tm_sw2h the same tensors with 128-row boxes.
+// tm_w2 / tm_sw2 use 256-row boxes, tm_w2h / tm_sw2h the same tensors with 128-row boxes;
+// tm_y (FP8 only; null: per-row stores) maps y [R, N] bf16 with 32-row x 64-column
+// 128B-swizzled boxes: the tiles then leave through shared memory and TMA stores.
 // The NVFP4 GEMMs for decode-sized groups (nvfp4_gemm_swap.cu): weights expanded
 // into TMEM as the MMA's A operand, a group's rows as N in 32-row chunks; maps
 // and parameters as for launch_nvfp4_gemm (p.mt_prefix not used).
@@ -210,7 +212,7 @@ cudaError_t launch_gemm_swap(const GemmParams& p, bool gemm1, int grid, const AM
                              const CUtensorMap& b1, const CUtensorMap& bs0, const CUtensorMap& bs1, cudaStream_t s);
 cudaError_t launch_gemm2(const GemmParams& p, bool fp8, bool pair, int grid, const AMaps& tm_a,
                          const CUtensorMap& tm_w2, const CUtensorMap& tm_w2h, const CUtensorMap& tm_sw2,
-                         const CUtensorMap& tm_sw2h, cudaStream_t s);
+                         const CUtensorMap& tm_sw2h, const CUtensorMap* tm_y, cudaStream_t s);
 cudaError_t launch_combine(const CombineParams& p, cudaStream_t s);
 // Expert parallelism: a rank's fp32 partial output, the sum of each token's
 // expert rows that this rank computed (pos < 0 left out), in slot order.

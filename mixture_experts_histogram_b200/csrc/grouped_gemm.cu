@@ -43,6 +43,10 @@
 // FP8: the fp32 block scales are not powers of two, so each 128-deep K block is
 // computed into a TMEM partial (two ping-pong buffers) and the epilogue warps
 // promote it into register accumulators with sa[row, kb] * sb[nblk, kb].
+// FP8 down GEMM with kStoreY: each epilogue warp writes its 32 rows x 128 bf16
+// columns of y into shared memory as two 128B-swizzled 32 x 64 boxes and one
+// lane stores them with TMA (whole 128-byte lines, asynchronously); the 64 KB
+// of staging take one pipeline stage (single: 3 stages, pair: 4).
 #include <cuda_bf16.h>
 #include <cuda_fp8.h>
 
@@ -66,16 +70,21 @@ constexpr int kScSlot = 132;                    // floats: 128 row scales + 2 bl
 #define MOE_FP8_CHUNK 16
 #endif
 constexpr int kFp8Chunk = MOE_FP8_CHUNK;        // TMEM columns per load when promoting FP8 partials
+constexpr int kYBox = 32 * 128;                 // bytes of one y store box: 32 rows x 64 bf16 columns
+constexpr int kYWarpBytes = 2 * kYBox;          // an epilogue warp's 32 rows x 128 columns
 
 
-template <bool kPair>
+// kStoreY: the FP8 down GEMM's bf16 y tiles leave through shared memory and TMA
+// stores (64 KB of staging, one fewer pipeline stage).
+template <bool kPair, bool kStoreY>
 struct Cfg {
-  static constexpr int kStages = kPair ? 6 : 4;
+  static constexpr int kStages = (kPair ? 6 : 4) - (kStoreY ? (kPair ? 2 : 1) : 0);
   static constexpr int kBBytes = (kPair ? 128 : 256) * kStageBytesK;  // this CTA's share of the B tile
   static constexpr int kStageBytes = kABytes + kBBytes;
   static constexpr int kTileRows = kPair ? 2 * kTileM : kTileM;      // rows of one work item
   static constexpr size_t kTiles = (size_t)kStages * kStageBytes;
-  static constexpr size_t kScales = kTiles;                           // float [kScRing][kScSlot]
+  static constexpr size_t kYStage = kTiles;                           // [kEpiWarps][2 boxes][32][128 B]
+  static constexpr size_t kScales = kYStage + (kStoreY ? kEpiWarps * kYWarpBytes : 0);  // float [kScRing][kScSlot]
   static constexpr size_t kBars = kScales + kScRing * kScSlot * 4;    // mbarriers (kNumBars x 8 bytes)
   static constexpr int kNumBars = 2 * kMaxStages + 2 + 2 + 1 + 2 * kScRing;
   static constexpr size_t kMisc = kBars + ((kNumBars * 8 + 127) / 128) * 128;  // tmem slot, abort flag
@@ -86,6 +95,7 @@ struct Cfg {
   static constexpr size_t kDynamic = kEnd + 1024;                     // + alignment slack
   static_assert(kMisc >= kBars + kNumBars * 8, "mbarriers overlap the misc words");
   static_assert(kDynamic <= 227 * 1024, "shared memory budget");
+  static_assert(kTiles % 1024 == 0, "the y staging boxes need 1024-byte alignment (128-byte swizzle)");
 };
 
 
@@ -108,12 +118,14 @@ struct BRows {
 };
 
 
-template <bool kFP8, bool kGemm1, bool kPair>
+template <bool kFP8, bool kGemm1, bool kPair, bool kStoreY>
 __global__ void __launch_bounds__(kThreads, 1)
     grouped_gemm_kernel(const GemmParams p, const __grid_constant__ AMaps tm_a,
                         const __grid_constant__ CUtensorMap tm_b0, const __grid_constant__ CUtensorMap tm_b1,
-                        const __grid_constant__ CUtensorMap tm_bs0, const __grid_constant__ CUtensorMap tm_bs1) {
-  using C = Cfg<kPair>;
+                        const __grid_constant__ CUtensorMap tm_bs0, const __grid_constant__ CUtensorMap tm_bs1,
+                        const __grid_constant__ CUtensorMap tm_y) {
+  static_assert(!kStoreY || (kFP8 && !kGemm1), "staged y stores belong to the FP8 down GEMM");
+  using C = Cfg<kPair, kStoreY>;
   constexpr int kElemsPerStage = kFP8 ? 128 : 64;  // 128 bytes of K per stage
   constexpr uint32_t kIdesc = idesc_mma(kFP8 ? 0u : 1u, kPair ? 2 * kTileM : kTileM, 256);
 
@@ -606,18 +618,41 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         } else {
           const float gw = row_ok ? (p.row_gate ? p.row_gate[row] : 1.0f) : 0.0f;
-          if (ok && row_ok && col_ok) {
+          auto packed = [&](int w) {  // y columns col0 + 8w .. +7 of this row, gated, bf16
+            const float2 a0 = acc[4 * w], a1 = acc[4 * w + 1], a2 = acc[4 * w + 2], a3 = acc[4 * w + 3];
+            return make_uint4(pack_bf16x2(a0.x * gw, a0.y * gw), pack_bf16x2(a1.x * gw, a1.y * gw),
+                              pack_bf16x2(a2.x * gw, a2.y * gw), pack_bf16x2(a3.x * gw, a3.y * gw));
+          };
+          // A warp whose 32 rows all lie inside the group writes them as two
+          // 32 x 64 boxes staged in shared memory (128B-swizzled) and stored by
+          // TMA, whole 128-byte lines; a thread-per-row store touches 32 lines
+          // per instruction. The warp straddling the group's end stores its
+          // rows from registers.
+          const int64_t wrow0 = (int64_t)it.row0 + my_off + q * 32;
+          if (kStoreY && ok && col_ok && wrow0 + 32 <= it.end) {
+            uint8_t* ys = smem + C::kYStage + (warp - 2) * kYWarpBytes;
+            if (lane == 0) bulk_wait_group_read0();  // the previous tile's boxes have been read
+            __syncwarp();
+#pragma unroll
+            for (int w = 0; w < 16; ++w)
+              *reinterpret_cast<uint4*>(ys + (w >> 3) * kYBox + lane * 128 + (((w & 7) ^ (lane & 7)) << 4)) =
+                  packed(w);
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              tma_store_2d(&tm_y, ys, col0, (int32_t)wrow0);
+              tma_store_2d(&tm_y, ys + kYBox, col0 + 64, (int32_t)wrow0);
+              bulk_commit_group();
+            }
+          } else if (ok && row_ok && col_ok) {
             uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.out) + row * p.N + col0);
 #pragma unroll
-            for (int w = 0; w < 16; ++w) {
-              const float2 a0 = acc[4 * w], a1 = acc[4 * w + 1], a2 = acc[4 * w + 2], a3 = acc[4 * w + 3];
-              dst[w] = make_uint4(pack_bf16x2(a0.x * gw, a0.y * gw), pack_bf16x2(a1.x * gw, a1.y * gw),
-                                  pack_bf16x2(a2.x * gw, a2.y * gw), pack_bf16x2(a3.x * gw, a3.y * gw));
-            }
+            for (int w = 0; w < 16; ++w) dst[w] = packed(w);
           }
         }
       }
     }
+    if (kStoreY && lane == 0) bulk_wait_group0();  // y boxes written before the CTA leaves
   }
 #ifdef MOE_DEBUG_STATE
   // Debug builds: each role's final counters, 16 ints per block from status[64],
@@ -643,20 +678,21 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-template <bool kFP8, bool kGemm1, bool kPair>
+template <bool kFP8, bool kGemm1, bool kPair, bool kStoreY = false>
 cudaError_t launch_one(const GemmParams& p, int grid, const AMaps& a, const CUtensorMap& b0,
-                       const CUtensorMap& b1, const CUtensorMap& bs0, const CUtensorMap& bs1, cudaStream_t s) {
-  auto kern = grouped_gemm_kernel<kFP8, kGemm1, kPair>;
+                       const CUtensorMap& b1, const CUtensorMap& bs0, const CUtensorMap& bs1, const CUtensorMap& y,
+                       cudaStream_t s) {
+  auto kern = grouped_gemm_kernel<kFP8, kGemm1, kPair, kStoreY>;
+  using C = Cfg<kPair, kStoreY>;
   static bool attr_set = false;  // per process; one device's limit serves every B200
   if (!attr_set) {
     cudaError_t e =
-        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Cfg<kPair>::kDynamic);
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::kDynamic);
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  if (!kPair) return launch_pdl(kern, dim3((unsigned)grid), dim3(kThreads), Cfg<kPair>::kDynamic, s, 1, p, a, b0, b1, bs0, bs1);
-  return launch_pdl(kern, dim3((unsigned)(grid & ~1)), dim3(kThreads), Cfg<kPair>::kDynamic, s, 2, p, a, b0, b1, bs0,
-                    bs1);
+  if (!kPair) return launch_pdl(kern, dim3((unsigned)grid), dim3(kThreads), C::kDynamic, s, 1, p, a, b0, b1, bs0, bs1, y);
+  return launch_pdl(kern, dim3((unsigned)(grid & ~1)), dim3(kThreads), C::kDynamic, s, 2, p, a, b0, b1, bs0, bs1, y);
 }
 
 }  // namespace
@@ -664,21 +700,27 @@ cudaError_t launch_one(const GemmParams& p, int grid, const AMaps& a, const CUte
 cudaError_t launch_gemm1(const GemmParams& p, bool fp8, bool pair, int grid, const AMaps& tm_a,
                          const CUtensorMap& tm_w1, const CUtensorMap& tm_w3, const CUtensorMap& tm_sw1,
                          const CUtensorMap& tm_sw3, cudaStream_t s) {
+  // (The y map is unused by the gate/up GEMM.)
   if (pair)
-    return fp8 ? launch_one<true, true, true>(p, grid, tm_a, tm_w1, tm_w3, tm_sw1, tm_sw3, s)
-               : launch_one<false, true, true>(p, grid, tm_a, tm_w1, tm_w3, tm_sw1, tm_sw3, s);
-  return fp8 ? launch_one<true, true, false>(p, grid, tm_a, tm_w1, tm_w3, tm_sw1, tm_sw3, s)
-             : launch_one<false, true, false>(p, grid, tm_a, tm_w1, tm_w3, tm_sw1, tm_sw3, s);
+    return fp8 ? launch_one<true, true, true>(p, grid, tm_a, tm_w1, tm_w3, tm_sw1, tm_sw3, tm_w1, s)
+               : launch_one<false, true, true>(p, grid, tm_a, tm_w1, tm_w3, tm_sw1, tm_sw3, tm_w1, s);
+  return fp8 ? launch_one<true, true, false>(p, grid, tm_a, tm_w1, tm_w3, tm_sw1, tm_sw3, tm_w1, s)
+             : launch_one<false, true, false>(p, grid, tm_a, tm_w1, tm_w3, tm_sw1, tm_sw3, tm_w1, s);
 }
 
 cudaError_t launch_gemm2(const GemmParams& p, bool fp8, bool pair, int grid, const AMaps& tm_a,
                          const CUtensorMap& tm_w2, const CUtensorMap& tm_w2h, const CUtensorMap& tm_sw2,
-                         const CUtensorMap& tm_sw2h, cudaStream_t s) {
+                         const CUtensorMap& tm_sw2h, const CUtensorMap* tm_y, cudaStream_t s) {
+  if (fp8 && tm_y) {
+    return pair ? launch_one<true, false, true, true>(p, grid, tm_a, tm_w2, tm_w2h, tm_sw2, tm_sw2h, *tm_y, s)
+                : launch_one<true, false, false, true>(p, grid, tm_a, tm_w2, tm_w2h, tm_sw2, tm_sw2h, *tm_y, s);
+  }
+  const CUtensorMap& unused = tm_w2;
   if (pair)
-    return fp8 ? launch_one<true, false, true>(p, grid, tm_a, tm_w2, tm_w2h, tm_sw2, tm_sw2h, s)
-               : launch_one<false, false, true>(p, grid, tm_a, tm_w2, tm_w2h, tm_sw2, tm_sw2h, s);
-  return fp8 ? launch_one<true, false, false>(p, grid, tm_a, tm_w2, tm_w2h, tm_sw2, tm_sw2h, s)
-             : launch_one<false, false, false>(p, grid, tm_a, tm_w2, tm_w2h, tm_sw2, tm_sw2h, s);
+    return fp8 ? launch_one<true, false, true>(p, grid, tm_a, tm_w2, tm_w2h, tm_sw2, tm_sw2h, unused, s)
+               : launch_one<false, false, true>(p, grid, tm_a, tm_w2, tm_w2h, tm_sw2, tm_sw2h, unused, s);
+  return fp8 ? launch_one<true, false, false>(p, grid, tm_a, tm_w2, tm_w2h, tm_sw2, tm_sw2h, unused, s)
+             : launch_one<false, false, false>(p, grid, tm_a, tm_w2, tm_w2h, tm_sw2, tm_sw2h, unused, s);
 }
 
 }  // namespace moe

@@ -80,10 +80,6 @@ struct NvLayout {
   static_assert(kMisc >= kBars + kNumBars * 8, "mbarriers overlap the misc words");
 };
 
-__device__ __forceinline__ void fence_proxy_async_smem() {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-
 template <bool kGemm1>
 __global__ void __launch_bounds__(kNvThreads, 1)
     nvfp4_gemm_kernel(const GemmParams p, const __grid_constant__ AMaps tm_a, const __grid_constant__ NvMaps tm) {

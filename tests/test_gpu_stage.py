@@ -122,6 +122,38 @@ def test_down_integer_inputs_bit_exact(m, fp8, variant):
     assert bad.size == 0, f"{len(bad)} outputs differ, first {bad[:4].tolist()}"
 
 
+def test_down_staged_stores_integer_inputs_bit_exact(m, variant):
+    """FP8 down GEMM with groups averaging a whole tile, so its y tiles leave
+    through shared memory and TMA stores: 32-row quarters wholly inside a group
+    are stored as boxes, the quarter straddling a group's end row by row (group
+    sizes 1, 300, 129, 256 and 200 put that end at every quarter offset). Rows
+    of one group written into the next would break the neighbour's sums."""
+    import torch
+    counts = [0, 1, 300, 129, 256, 200]
+    cfg, dev, (_, _, w2), *_ = _setup(m, True)
+    offsets = np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
+    R = int(offsets[-1])
+    assert R >= 128 * (E + 1)
+    group = np.repeat(np.arange(E + 1), counts)
+    ws = torch.empty(m.moe_workspace_bytes(cfg, -(-R // 3)), dtype=torch.uint8, device="cuda")
+    a = _ints(7, (R, I))
+    gate = np.random.default_rng(8).choice(np.array([0.25, 0.5, 1.0, 2.0], np.float32), size=R)
+    y = torch.full((R, H), float("nan"), dtype=torch.bfloat16, device="cuda")
+    m.moe_grouped_gemm(cfg, m.MOE_STAGE_DOWN, R, m.to_device(offsets), m.to_device(_codes(a, True)),
+                       m.to_device(np.ones((R, I // 128), np.float32)), m.make_weights(dev), y, ws,
+                       row_gate=m.to_device(gate))
+    assert m.moe_read_status(ws) == 0
+    got = y.view(torch.int16).cpu().numpy().view(np.uint16)
+    ref = np.empty((R, H), np.float64)
+    for g in range(E + 1):
+        rr = group == g
+        ref[rr] = (a[rr] @ w2[g].T).astype(np.float64)
+    ref *= gate[:, None].astype(np.float64)
+    want = synth.f32_to_bf16(ref.astype(np.float32))
+    bad = np.argwhere(got != want)
+    assert bad.size == 0, f"{len(bad)} outputs differ, first {bad[:4].tolist()}"
+
+
 @pytest.mark.parametrize("fp8", [True, False], ids=["fp8", "bf16"])
 def test_down_split_k_integer_inputs_bit_exact(m, fp8, variant):
     """One group of 50 rows under a 64-row call, K = 2048, H = 512: two output
