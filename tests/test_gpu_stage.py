@@ -99,6 +99,52 @@ def test_gate_up_integer_inputs_bit_exact(m, fp8, variant):
     assert bad.size == 0, f"{len(bad)} sums differ, first {bad[:4].tolist()}"
 
 
+def test_gate_up_h_codes_bit_exact(m, variant):
+    """FP8 gate/up GEMM through SwiGLU and the 1x128 quantisation of h, on
+    inputs that make every step exact: positive activations and W1 = 1 put each
+    gate sum at 512..1024, where exp(-g) underflows and silu(g) = g exactly in
+    fp32, and g * u stays an integer below 2^24. The codes then follow from the
+    block quantisation alone (scale = amax/448, codes = E4M3 of h * (1/scale),
+    ties to even, saturating), for every row position of a tile, including the
+    ragged ends of groups."""
+    import torch
+    cfg, _, _, offsets, R, group, ws = _setup(m, True)
+    rng = np.random.default_rng(21)
+    a = rng.integers(1, 3, size=(R, H)).astype(np.int64)
+    w1 = np.ones((E + 1, I, H), np.int64)
+    w3 = rng.integers(-2, 3, size=(E + 1, I, H)).astype(np.int64)
+    host = {"router_w": synth.normal_bf16(0, 1, (E, H), 0.05), "router_bias": None,
+            "w1": _codes(w1[:E], True), "w3": _codes(w3[:E], True), "w2": _codes(np.ones((E, H, I)), True),
+            "sw1": _codes(w1[E:], True), "sw3": _codes(w3[E:], True), "sw2": _codes(np.ones((1, H, I)), True)}
+    for k, shp in (("s1", (E, I // 128, H // 128)), ("s3", (E, I // 128, H // 128)), ("s2", (E, H // 128, I // 128)),
+                   ("ss1", (1, I // 128, H // 128)), ("ss3", (1, I // 128, H // 128)),
+                   ("ss2", (1, H // 128, I // 128))):
+        host[k] = np.ones(shp, np.float32)
+    dev = m.upload_weights(host)
+    h = torch.zeros((R, I), dtype=torch.uint8, device="cuda")
+    hs = torch.zeros((R, I // 128), dtype=torch.float32, device="cuda")
+    m.moe_grouped_gemm(cfg, m.MOE_STAGE_GATE_UP, R, m.to_device(offsets), m.to_device(_codes(a, True)),
+                       m.to_device(np.ones((R, H // 128), np.float32)), m.make_weights(dev), h, ws, out_scale=hs)
+    assert m.moe_read_status(ws) == 0
+    hv = np.empty((R, I), np.float64)
+    for g in range(E + 1):
+        rr = group == g
+        gs, us = a[rr] @ w1[g].T, a[rr] @ w3[g].T
+        assert gs.size == 0 or gs.min() >= 512
+        hv[rr] = (gs * us).astype(np.float64)
+    assert np.abs(hv).max() < 2 ** 24
+    hb = hv.astype(np.float32).reshape(R, I // 128, 128)
+    amax = np.abs(hb).max(axis=2)
+    scale = np.where(amax > 0, amax / np.float32(448), np.float32(1)).astype(np.float32)
+    inv = np.where(amax > 0, np.float32(1) / scale, np.float32(0)).astype(np.float32)
+    want = oracle.e4m3_encode((hb * inv[:, :, None]).astype(np.float32)).reshape(R, I)
+    got_s = hs.cpu().numpy()
+    assert np.array_equal(got_s.view(np.uint32), scale.view(np.uint32))
+    got = h.cpu().numpy()
+    bad = np.argwhere(got != want)
+    assert bad.size == 0, f"{len(bad)} codes differ, first {bad[:4].tolist()}"
+
+
 @pytest.mark.parametrize("fp8", [True, False], ids=["fp8", "bf16"])
 def test_down_integer_inputs_bit_exact(m, fp8, variant):
     import torch
