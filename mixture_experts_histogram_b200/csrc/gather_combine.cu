@@ -40,9 +40,10 @@ __global__ void __launch_bounds__(256) gather_bf16_kernel(const GatherParams p) 
 
 // One half-warp per 128-element block: each lane loads 8 bf16 (16 bytes),
 // the half-warp reduces the block's amax, and each lane stores its 8 codes
-// (8 bytes) to every destination row.
+// (8 bytes) to every destination row. Six CTAs' registers per SM leave room
+// for the next kernel's CTAs to start under programmatic dependent launch.
 template <int kMaxSlots>
-__global__ void __launch_bounds__(256) gather_fp8_kernel(const GatherParams p) {
+__global__ void __launch_bounds__(256, 6) gather_fp8_kernel(const GatherParams p) {
   pdl_wait();
   pdl_trigger();
   const int64_t t = blockIdx.x;
@@ -52,44 +53,52 @@ __global__ void __launch_bounds__(256) gather_fp8_kernel(const GatherParams p) {
   int32_t rows[kMaxSlots];  // destination rows (< 2^31)
 #pragma unroll
   for (int j = 0; j < kMaxSlots; ++j) rows[j] = j < p.S ? (p.pos ? p.pos[t * p.S + j] : (int32_t)t) : -1;
-  for (int kb0 = 2 * warp; kb0 < nblk; kb0 += 16) {
-    const int kb = kb0 + half;
-    const bool active = kb < nblk;
-    uint4 raw = make_uint4(0, 0, 0, 0);
-    if (active) raw = __ldcs(reinterpret_cast<const uint4*>(p.x + t * p.H + kb * 128) + hl);
-    const __nv_bfloat162* b = reinterpret_cast<const __nv_bfloat162*>(&raw);
-    float f[8];
+  // Two blocks per half-warp and pass, both loads issued before either is used.
+  for (int kb00 = 2 * warp; kb00 < nblk; kb00 += 32) {
+    uint4 raws[2];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const float2 v = __bfloat1622float2(b[i]);
-      f[2 * i] = v.x;
-      f[2 * i + 1] = v.y;
+    for (int u = 0; u < 2; ++u) {
+      const int kb = kb00 + 16 * u + half;
+      raws[u] = kb < nblk ? __ldcs(reinterpret_cast<const uint4*>(p.x + t * p.H + kb * 128) + hl)
+                          : make_uint4(0, 0, 0, 0);
     }
-    float amax = 0.0f;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(f[i]));
+    for (int u = 0; u < 2; ++u) {
+      const int kb = kb00 + 16 * u + half;
+      const __nv_bfloat162* b = reinterpret_cast<const __nv_bfloat162*>(&raws[u]);
+      float f[8];
 #pragma unroll
-    for (int off = 8; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
-    float s = 1.0f;
-    uint2 codes = make_uint2(0, 0);
-    if (amax > 0.0f) {
-      s = __fdiv_rn(amax, 448.0f);
-      uint32_t w[4];
+      for (int i = 0; i < 4; ++i) {
+        const float2 v = __bfloat1622float2(b[i]);
+        f[2 * i] = v.x;
+        f[2 * i + 1] = v.y;
+      }
+      float amax = 0.0f;
 #pragma unroll
-      for (int i = 0; i < 4; ++i)
-        w[i] = __nv_cvt_float2_to_fp8x2(make_float2(__fdiv_rn(f[2 * i], s), __fdiv_rn(f[2 * i + 1], s)),
-                                        __NV_SATFINITE, __NV_E4M3);
-      codes = make_uint2(w[0] | (w[1] << 16), w[2] | (w[3] << 16));
-    }
-    if (!active) continue;
+      for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(f[i]));
 #pragma unroll
-    for (int j = 0; j < kMaxSlots; ++j) {
-      const int64_t row = rows[j];
-      if (row < 0) continue;
-      *reinterpret_cast<uint2*>(static_cast<uint8_t*>(p.xp) + row * p.H + kb * 128 + hl * 8) = codes;
-      if (hl == 0) {
-        if (p.scale_row_major) p.sxp[row * nblk + kb] = s;
-        else p.sxp[(int64_t)kb * p.rows_pad + row] = s;
+      for (int off = 8; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+      float s = 1.0f;
+      uint2 codes = make_uint2(0, 0);
+      if (amax > 0.0f) {
+        s = __fdiv_rn(amax, 448.0f);
+        uint32_t w[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          w[i] = __nv_cvt_float2_to_fp8x2(make_float2(__fdiv_rn(f[2 * i], s), __fdiv_rn(f[2 * i + 1], s)),
+                                          __NV_SATFINITE, __NV_E4M3);
+        codes = make_uint2(w[0] | (w[1] << 16), w[2] | (w[3] << 16));
+      }
+      if (kb >= nblk) continue;
+#pragma unroll
+      for (int j = 0; j < kMaxSlots; ++j) {
+        const int64_t row = rows[j];
+        if (row < 0) continue;
+        *reinterpret_cast<uint2*>(static_cast<uint8_t*>(p.xp) + row * p.H + kb * 128 + hl * 8) = codes;
+        if (hl == 0) {
+          if (p.scale_row_major) p.sxp[row * nblk + kb] = s;
+          else p.sxp[(int64_t)kb * p.rows_pad + row] = s;
+        }
       }
     }
   }
