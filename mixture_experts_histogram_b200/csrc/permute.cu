@@ -12,7 +12,7 @@
 //   2. scan: one CTA scans chunk counts per expert (one warp per expert), then
 //      the expert totals -> counts, offsets, and the per-group prefixes of
 //      128-row tiles and 256-row pair tiles the grouped GEMMs schedule from;
-//      chunk_base becomes absolute row bases.
+//      chunk_base becomes each chunk's base inside its group.
 //   3. scatter: each warp ranks its 32 tokens' pairs in (token, slot) order
 //      with __match_any_sync (equal experts in one 32-pair round rank by lane),
 //      warps are then offset by an exclusive scan over the CTA's 8 warps, and
@@ -59,20 +59,42 @@ __device__ __forceinline__ int warp_inclusive_scan(int v, int lane) {
   return v;
 }
 
-__device__ __forceinline__ void scan_block(const PermuteParams& p, int* cnt_s, int* off_s) {
+__device__ __forceinline__ void scan_block(const PermuteParams& p, int* cnt_s) {
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32, nwarps = blockDim.x / 32;
-  // per-expert exclusive scan over chunks (bases relative to the expert)
-  for (int e = warp; e < p.E; e += nwarps) {
-    int running = 0;
-    int32_t* row = p.chunk_base + (int64_t)e * p.chunks;
-    for (int c0 = 0; c0 < p.chunks; c0 += 32) {
-      const int c = c0 + lane;
-      const int v = c < p.chunks ? row[c] : 0;
-      const int incl = warp_inclusive_scan(v, lane);
-      if (c < p.chunks) row[c] = running + incl - v;
-      running += __shfl_sync(0xffffffffu, incl, 31);
+  // per-expert exclusive scan over chunks (bases relative to the expert's
+  // first row). Up to 32 chunks (T <= 8192): a warp loads the counts of 12
+  // experts before scanning any, so their load latencies overlap.
+  if (p.chunks <= 32) {
+    constexpr int kBatch = 12;
+    for (int e0 = warp; e0 < p.E; e0 += nwarps * kBatch) {
+      int v[kBatch];
+#pragma unroll
+      for (int j = 0; j < kBatch; ++j) {
+        const int e = e0 + nwarps * j;
+        v[j] = (e < p.E && lane < p.chunks) ? p.chunk_base[(int64_t)e * p.chunks + lane] : 0;
+      }
+#pragma unroll
+      for (int j = 0; j < kBatch; ++j) {
+        const int e = e0 + nwarps * j;
+        const int incl = warp_inclusive_scan(v[j], lane);
+        if (e < p.E && lane < p.chunks) p.chunk_base[(int64_t)e * p.chunks + lane] = incl - v[j];
+        const int total = __shfl_sync(0xffffffffu, incl, 31);
+        if (e < p.E && lane == 0) cnt_s[e] = total;
+      }
     }
-    if (lane == 0) cnt_s[e] = running;
+  } else {
+    for (int e = warp; e < p.E; e += nwarps) {
+      int running = 0;
+      int32_t* row = p.chunk_base + (int64_t)e * p.chunks;
+      for (int c0 = 0; c0 < p.chunks; c0 += 32) {
+        const int c = c0 + lane;
+        const int v = c < p.chunks ? row[c] : 0;
+        const int incl = warp_inclusive_scan(v, lane);
+        if (c < p.chunks) row[c] = running + incl - v;
+        running += __shfl_sync(0xffffffffu, incl, 31);
+      }
+      if (lane == 0) cnt_s[e] = running;
+    }
   }
   if (threadIdx.x == 0 && p.S) cnt_s[p.E] = p.sh_t1 - p.sh_t0;
   __syncthreads();
@@ -92,7 +114,6 @@ __device__ __forceinline__ void scan_block(const PermuteParams& p, int* cnt_s, i
         p.offsets[g] = run_off + ic - c;
         p.mt_prefix[g] = run_mt + im - mt;
         p.mp_prefix[g] = run_mp + ip - mp;
-        off_s[g] = run_off + ic - c;
       }
       run_off += __shfl_sync(0xffffffffu, ic, 31);
       run_mt += __shfl_sync(0xffffffffu, im, 31);
@@ -105,16 +126,13 @@ __device__ __forceinline__ void scan_block(const PermuteParams& p, int* cnt_s, i
     }
   }
   __syncthreads();
-  const int64_t n = (int64_t)p.E * p.chunks;
-  for (int64_t i = threadIdx.x; i < n; i += blockDim.x) p.chunk_base[i] += off_s[i / p.chunks];
 }
 
 __global__ void __launch_bounds__(1024) scan_kernel(const PermuteParams p) {
   pdl_wait();
   pdl_trigger();
   __shared__ int cnt_s[kMaxExperts + 1];
-  __shared__ int off_s[kMaxExperts + 2];
-  scan_block(p, cnt_s, off_s);
+  scan_block(p, cnt_s);
 }
 
 __device__ __forceinline__ void scatter_block(const PermuteParams& p, int chunk, int (*wcnt)[kMaxExperts]) {
@@ -151,9 +169,10 @@ __device__ __forceinline__ void scatter_block(const PermuteParams& p, int chunk,
     }
   }
   __syncthreads();
-  // Pass 2: warp offsets per expert, on top of this chunk's absolute base.
+  // Pass 2: warp offsets per expert, on top of this chunk's base (the group's
+  // first row plus the chunk's base inside the group).
   for (int e = threadIdx.x; e < p.E; e += blockDim.x) {
-    int run = p.chunk_base[(int64_t)e * p.chunks + chunk];
+    int run = p.offsets[e] + p.chunk_base[(int64_t)e * p.chunks + chunk];
 #pragma unroll
     for (int w = 0; w < 8; ++w) {
       const int v = wcnt[w][e];
@@ -240,7 +259,7 @@ __global__ void __launch_bounds__(256) permute_one_chunk_kernel(const PermutePar
         p.offsets[g] = run_off + ic - c;
         p.mt_prefix[g] = run_mt + im - mt;
         p.mp_prefix[g] = run_mp + ip - mp;
-        if (g < p.E) p.chunk_base[g] = run_off + ic - c;  // the one chunk starts at the group's offset
+        if (g < p.E) p.chunk_base[g] = 0;  // the one chunk starts at its group's first row
       }
       run_off += __shfl_sync(0xffffffffu, ic, 31);
       run_mt += __shfl_sync(0xffffffffu, im, 31);

@@ -218,21 +218,22 @@ __global__ void __launch_bounds__(kRouterThreads, 1)
 
 // One warp per token: sum the K-split partial logits in split order, add the
 // bias, pick the top k (largest logit first, ties to the lower index), and
-// renormalise their softmax probabilities.
+// renormalise their softmax probabilities. kPer: experts per lane (E <= 32
+// kPer); kSplitBatch: K splits whose loads are issued together. Both are sized
+// to the call so the kernel keeps few registers (more warps in flight).
+template <int kPer, int kSplitBatch>
 __global__ void __launch_bounds__(256) topk_kernel(const TopkParams p) {
   pdl_wait();
   pdl_trigger();
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int64_t t = (int64_t)blockIdx.x * 8 + warp;
   if (t >= p.T) return;
-  constexpr int kPer = kMaxExperts / 32;
   float l[kPer];
-  // The loads of up to four splits are independent and issued together; the
+  // The loads of a batch of splits are independent and issued together; the
   // splits are added in split order.
   const float* __restrict__ part = p.partial;
 #pragma unroll
   for (int i = 0; i < kPer; ++i) l[i] = (lane + 32 * i < p.E) ? 0.0f : -INFINITY;
-  constexpr int kSplitBatch = 4;
   for (int s0 = 0; s0 < p.ksplit; s0 += kSplitBatch) {
     float v[kSplitBatch][kPer];
 #pragma unroll
@@ -320,8 +321,21 @@ cudaError_t launch_router_gemm(const RouterParams& p, const CUtensorMap& tm_x, c
   return launch_pdl(router_gemm_kernel, grid, dim3(kRouterThreads), smem, s, 1, p, tm_x, tm_w);
 }
 
+namespace {
+template <int kPer>
+cudaError_t launch_topk_per(const TopkParams& p, cudaStream_t s) {
+  const dim3 grid((unsigned)ceil_div(p.T, 8));
+  if (p.ksplit <= 2) return launch_pdl(topk_kernel<kPer, 2>, grid, dim3(256), 0, s, 1, p);
+  return launch_pdl(topk_kernel<kPer, 4>, grid, dim3(256), 0, s, 1, p);
+}
+}  // namespace
+
 cudaError_t launch_topk(const TopkParams& p, cudaStream_t s) {
-  return launch_pdl(topk_kernel, dim3((unsigned)ceil_div(p.T, 8)), dim3(256), 0, s, 1, p);
+  static_assert(kMaxExperts <= 16 * 32, "top-k lanes hold at most 16 experts each");
+  if (p.E <= 4 * 32) return launch_topk_per<4>(p, s);
+  if (p.E <= 8 * 32) return launch_topk_per<8>(p, s);
+  if (p.E <= 12 * 32) return launch_topk_per<12>(p, s);
+  return launch_topk_per<16>(p, s);
 }
 
 }  // namespace moe
