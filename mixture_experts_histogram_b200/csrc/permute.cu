@@ -135,28 +135,40 @@ __global__ void __launch_bounds__(1024) scan_kernel(const PermuteParams p) {
   scan_block(p, cnt_s);
 }
 
-__device__ __forceinline__ void scatter_block(const PermuteParams& p, int chunk, int (*wcnt)[kMaxExperts]) {
+// off_s: the G + 1 group offsets in shared memory, filled by the caller before
+// the block barrier inside.
+__device__ __forceinline__ void scatter_block(const PermuteParams& p, int chunk, int (*wcnt)[kMaxExperts],
+                                              const int* off_s) {
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  for (int i = threadIdx.x; i < 8 * kMaxExperts; i += blockDim.x) (&wcnt[0][0])[i] = 0;
-  __syncthreads();
-
   const int64_t tw0 = (int64_t)chunk * kHistChunk + warp * 32;  // this warp's first token
   int rank[kMaxTopK];
   int ekeep[kMaxTopK];
-  // Pass 1: ranks inside the warp, pairs taken in (token, slot) order, 32 per round.
+  float gkeep[kMaxTopK];
+  // The pairs' experts and gates, all loaded before they are used.
 #pragma unroll
   for (int r = 0; r < kMaxTopK; ++r) {
     ekeep[r] = -1;
-    rank[r] = 0;
+    gkeep[r] = 0.0f;
     if (r < p.k) {
       const int pidx = r * 32 + lane;
       const int64_t t = tw0 + pidx / p.k;
       const int j = pidx % p.k;
-      int e = -1;
       if (t < p.T) {
-        e = p.idx[t * p.k + j] - p.e0;  // this call's group; others are left out
-        if (e < 0 || e >= p.E || e + p.e0 >= p.E_all) e = -1;
+        ekeep[r] = p.idx[t * p.k + j] - p.e0;  // this call's group; others are left out
+        if (p.row_gate) gkeep[r] = p.gate[t * p.k + j];
       }
+    }
+  }
+  for (int i = threadIdx.x; i < 8 * kMaxExperts; i += blockDim.x) (&wcnt[0][0])[i] = 0;
+  __syncthreads();
+
+  // Pass 1: ranks inside the warp, pairs taken in (token, slot) order, 32 per round.
+#pragma unroll
+  for (int r = 0; r < kMaxTopK; ++r) {
+    rank[r] = 0;
+    if (r < p.k) {
+      int e = ekeep[r];
+      if (e < 0 || e >= p.E || e + p.e0 >= p.E_all) e = -1;
       const int key = e >= 0 ? e : (0x40000000 + lane);  // unmatched sentinel for empty lanes
       const unsigned m = __match_any_sync(0xffffffffu, key);
       const int rk = __popc(m & ((1u << lane) - 1u));
@@ -172,7 +184,7 @@ __device__ __forceinline__ void scatter_block(const PermuteParams& p, int chunk,
   // Pass 2: warp offsets per expert, on top of this chunk's base (the group's
   // first row plus the chunk's base inside the group).
   for (int e = threadIdx.x; e < p.E; e += blockDim.x) {
-    int run = p.offsets[e] + p.chunk_base[(int64_t)e * p.chunks + chunk];
+    int run = off_s[e] + p.chunk_base[(int64_t)e * p.chunks + chunk];
 #pragma unroll
     for (int w = 0; w < 8; ++w) {
       const int v = wcnt[w][e];
@@ -195,7 +207,7 @@ __device__ __forceinline__ void scatter_block(const PermuteParams& p, int chunk,
           const int row = wcnt[warp][e] + rank[r];
           p.perm[row] = (int32_t)t;
           p.pos[t * S + j] = row;
-          if (p.row_gate) p.row_gate[row] = p.gate[t * p.k + j];
+          if (p.row_gate) p.row_gate[row] = gkeep[r];
         } else {
           p.pos[t * S + j] = -1;  // a pair left out (another rank's expert, or a bad index)
         }
@@ -207,7 +219,7 @@ __device__ __forceinline__ void scatter_block(const PermuteParams& p, int chunk,
     const int64_t t = (int64_t)chunk * kHistChunk + threadIdx.x;
     if (t < p.T) {
       if (t >= p.sh_t0 && t < p.sh_t1) {
-        const int row = p.offsets[p.E] + (int)(t - p.sh_t0);
+        const int row = off_s[p.E] + (int)(t - p.sh_t0);
         p.perm[row] = (int32_t)t;
         p.pos[t * S + p.k] = row;
         if (p.row_gate) p.row_gate[row] = 1.0f;
@@ -218,21 +230,24 @@ __device__ __forceinline__ void scatter_block(const PermuteParams& p, int chunk,
   }
 }
 
-__global__ void __launch_bounds__(256) scatter_kernel(const PermuteParams p) {
+__global__ void __launch_bounds__(256, 1) scatter_kernel(const PermuteParams p) {
   pdl_wait();
   pdl_trigger();
   __shared__ int wcnt[8][kMaxExperts];
-  scatter_block(p, blockIdx.x, wcnt);
+  __shared__ int off_s[kMaxExperts + 2];
+  for (int g = threadIdx.x; g <= p.G; g += blockDim.x) off_s[g] = p.offsets[g];
+  scatter_block(p, blockIdx.x, wcnt, off_s);
 }
 
 // T <= 256: the three steps in one CTA. With a single chunk the per-expert
 // chunk scan is the identity, so the counts come straight from the shared
-// histogram, one warp scans them over the groups, and the scatter follows. The
-// block barriers also make each step's global writes visible to the next.
-__global__ void __launch_bounds__(256) permute_one_chunk_kernel(const PermuteParams p) {
+// histogram, the block scans them over the groups, and the scatter follows.
+__global__ void __launch_bounds__(256, 1) permute_one_chunk_kernel(const PermuteParams p) {
   pdl_wait();
   pdl_trigger();
   __shared__ int wcnt[8][kMaxExperts];  // scatter; rows 0-1 first hold the expert counts
+  __shared__ int off_s[kMaxExperts + 2];
+  __shared__ int wtot[3][8];
   int* cnt = &wcnt[0][0];
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   for (int e = threadIdx.x; e < p.E; e += blockDim.x) cnt[e] = 0;
@@ -244,35 +259,59 @@ __global__ void __launch_bounds__(256) permute_one_chunk_kernel(const PermutePar
     else if (e >= 0 && e < p.E) atomicAdd(&cnt[e], 1);
   }
   __syncthreads();
-  if (warp == 0) {
-    int run_off = 0, run_mt = 0, run_mp = 0;
-    for (int g0 = 0; g0 < p.G; g0 += 32) {
-      const int g = g0 + lane;
-      const int c = g < p.E ? cnt[g] : (g < p.G ? p.sh_t1 - p.sh_t0 : 0);  // group E: the shared expert
-      const int mt = (c + kTileM - 1) / kTileM;
-      const int mp = (c + 2 * kTileM - 1) / (2 * kTileM);
-      const int ic = warp_inclusive_scan(c, lane);
-      const int im = warp_inclusive_scan(mt, lane);
-      const int ip = warp_inclusive_scan(mp, lane);
-      if (g < p.G) {
-        p.counts[g] = c;
-        p.offsets[g] = run_off + ic - c;
-        p.mt_prefix[g] = run_mt + im - mt;
-        p.mp_prefix[g] = run_mp + ip - mp;
-        if (g < p.E) p.chunk_base[g] = 0;  // the one chunk starts at its group's first row
-      }
-      run_off += __shfl_sync(0xffffffffu, ic, 31);
-      run_mt += __shfl_sync(0xffffffffu, im, 31);
-      run_mp += __shfl_sync(0xffffffffu, ip, 31);
-    }
-    if (lane == 0) {
-      p.offsets[p.G] = run_off;
-      p.mt_prefix[p.G] = run_mt;
-      p.mp_prefix[p.G] = run_mp;
-    }
+  // Exclusive scans over the G groups of their rows, 128-row tiles and 256-row
+  // pair tiles: kPer consecutive groups per thread, a warp scan of the
+  // threads' sums, then the warps' totals.
+  constexpr int kPer = (kMaxExperts + 1 + 255) / 256;
+  int c[kPer], mt[kPer], mp[kPer];
+  int sc = 0, sm = 0, sp = 0;
+#pragma unroll
+  for (int u = 0; u < kPer; ++u) {
+    const int g = threadIdx.x * kPer + u;
+    c[u] = g < p.E ? cnt[g] : (g < p.G ? p.sh_t1 - p.sh_t0 : 0);  // group E: the shared expert
+    mt[u] = (c[u] + kTileM - 1) / kTileM;
+    mp[u] = (c[u] + 2 * kTileM - 1) / (2 * kTileM);
+    sc += c[u];
+    sm += mt[u];
+    sp += mp[u];
+  }
+  const int ic = warp_inclusive_scan(sc, lane);
+  const int im = warp_inclusive_scan(sm, lane);
+  const int ip = warp_inclusive_scan(sp, lane);
+  if (lane == 31) {
+    wtot[0][warp] = ic;
+    wtot[1][warp] = im;
+    wtot[2][warp] = ip;
   }
   __syncthreads();
-  scatter_block(p, 0, wcnt);
+  int run_off = ic - sc, run_mt = im - sm, run_mp = ip - sp;
+  for (int w = 0; w < warp; ++w) {
+    run_off += wtot[0][w];
+    run_mt += wtot[1][w];
+    run_mp += wtot[2][w];
+  }
+#pragma unroll
+  for (int u = 0; u < kPer; ++u) {
+    const int g = threadIdx.x * kPer + u;
+    if (g < p.G) {
+      p.counts[g] = c[u];
+      p.offsets[g] = run_off;
+      p.mt_prefix[g] = run_mt;
+      p.mp_prefix[g] = run_mp;
+      off_s[g] = run_off;
+      if (g < p.E) p.chunk_base[g] = 0;  // the one chunk starts at its group's first row
+    } else if (g == p.G) {
+      p.offsets[g] = run_off;
+      p.mt_prefix[g] = run_mt;
+      p.mp_prefix[g] = run_mp;
+      off_s[g] = run_off;
+    }
+    run_off += c[u];
+    run_mt += mt[u];
+    run_mp += mp[u];
+  }
+  __syncthreads();
+  scatter_block(p, 0, wcnt, off_s);
 }
 
 // Tile prefixes of caller-given group offsets (the grouped-GEMM stage entry
