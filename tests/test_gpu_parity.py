@@ -125,10 +125,12 @@ def test_route_parity(m, shape):
 
 # ------------------------------------------------------- histogram/permute --
 
-# T <= 256 runs the one-launch path (one 256-token chunk), larger T the three kernels.
+# T <= 256 runs the one-launch path (one 256-token chunk), larger T the three
+# kernels, whose chunk scan batches its loads up to 32 chunks (T <= 8192) and
+# loops over the chunks beyond.
 PERMUTE_CASES = [(32, 16, 2, 1), (1000, 352, 8, 1), (8192, 352, 8, 1), (777, 352, 8, 0), (1, 352, 8, 1),
                  (4096, 512, 16, 1), (300, 5, 5, 1), (64, 352, 8, 1), (256, 512, 16, 1), (255, 352, 8, 0),
-                 (257, 352, 8, 1)]
+                 (257, 352, 8, 1), (8193, 352, 8, 1), (12345, 100, 6, 1), (32768, 352, 8, 1), (40000, 352, 8, 1)]
 
 
 @pytest.mark.parametrize("T,E,k,S", PERMUTE_CASES)
