@@ -79,6 +79,51 @@ def test_quantize_act_bit_exact(m):
     assert bad.size == 0, f"{len(bad)} codes differ, first {bad[:5].tolist()}"
 
 
+def _quant_blocks_every_bf16_and_e4m3_tie():
+    """Blocks of 128 bf16 values: every finite bf16 bit pattern, in order (blocks
+    of one exponent) and shuffled (blocks spanning many exponents); and for block
+    maxima 448 * 2^k, the E4M3 midpoints and values times 2^k, so that x / scale
+    lands exactly on every rounding tie and representable value."""
+    pats = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    finite = pats[(pats & 0x7F80) != 0x7F80]
+    rng = np.random.default_rng(77)
+    blocks = [finite, rng.permutation(finite)]
+    vals = np.unique(oracle.e4m3_decode(np.arange(256, dtype=np.uint8)))
+    pos = vals[np.isfinite(vals) & (vals > 0)].astype(np.float64)
+    mids = (pos[:-1] + pos[1:]) / 2
+    cand = np.concatenate([mids, pos, -mids, -pos])
+    for k in range(-30, 31):
+        xs = cand * 2.0 ** k
+        for c0 in range(0, len(xs), 127):
+            blk = np.zeros(128, np.float32)
+            blk[0] = 448.0 * 2.0 ** k
+            chunk = xs[c0:c0 + 127].astype(np.float32)
+            blk[1:1 + len(chunk)] = chunk
+            b = synth.f32_to_bf16(blk)
+            assert np.array_equal((b.astype(np.uint32) << 16).view(np.float32), blk)  # exact in bf16
+            blocks.append(b)
+    flat = np.concatenate(blocks)
+    flat = np.concatenate([flat, np.zeros((-len(flat)) % 4096, np.uint16)])
+    return flat.reshape(-1, 4096)
+
+
+def test_quantize_act_every_bf16_and_e4m3_tie(m):
+    """The activation quantisation over every finite bf16 value and every E4M3
+    rounding tie (x / scale exactly halfway between two codes), bit-exact against
+    the oracle's IEEE division and round-to-nearest-even."""
+    import torch
+    x = _quant_blocks_every_bf16_and_e4m3_tie()
+    T = x.shape[0]
+    q_ref, s_ref = oracle.quantize_rows(x)
+    q = torch.empty((T, 4096), dtype=torch.uint8, device="cuda")
+    s = torch.empty((T, 32), dtype=torch.float32, device="cuda")
+    m.moe_quantize_act(T, 4096, m.to_device(x), q, s)
+    torch.cuda.synchronize()
+    assert np.array_equal(s.cpu().numpy().view(np.uint32), s_ref.view(np.uint32))
+    bad = np.argwhere(q.cpu().numpy() != q_ref)
+    assert bad.size == 0, f"{len(bad)} codes differ, first {bad[:5].tolist()}"
+
+
 # ------------------------------------------------------------------ routing --
 
 ROUTE_CASES = [
