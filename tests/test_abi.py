@@ -191,3 +191,26 @@ def test_product_path_does_not_touch_the_oracle():
             if f.endswith((".py", ".cu", ".cuh", ".h")):
                 src = open(os.path.join(dirpath, f)).read()
                 assert "import oracle" not in src and "from oracle" not in src and "orc_" not in src, f
+
+
+def test_traffic_hash_covers_every_grouped_gemm_source():
+    """bench.py drops a stored DRAM-traffic figure once the sources it was taken on
+    change; every file the grouped-GEMM sources include (and the launch code that
+    builds their tensor maps) must be part of that hash."""
+    import sys
+    sys.path.insert(0, ROOT)
+    import bench
+    csrc = os.path.join(ROOT, "mixture_experts_histogram_b200", "csrc")
+    gemm = [f for f in os.listdir(csrc) if f.endswith(".cu") and "gemm" in f]
+    assert gemm and set(gemm) <= set(bench.GEMM_SOURCES)
+    todo, seen = list(gemm), set()
+    while todo:
+        f = todo.pop()
+        if f in seen:
+            continue
+        seen.add(f)
+        for inc in re.findall(r'#include\s+"([^"]+)"', open(os.path.join(csrc, f)).read()):
+            if os.path.exists(os.path.join(csrc, inc)):
+                todo.append(inc)
+    assert seen <= set(bench.GEMM_SOURCES), sorted(seen - set(bench.GEMM_SOURCES))
+    assert "abi.cu" in bench.GEMM_SOURCES
